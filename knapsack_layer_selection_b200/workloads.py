@@ -1,0 +1,203 @@
+"""Synthetic KnapSpec workloads: configuration records and seeded input draws.
+
+This module only describes shapes and draws seeded random numbers.  It holds no
+arithmetic of the method (no norm, attention, MLP, cosine, quantisation, DP or
+TPT); both the CUDA library's callers and the CPU oracle's callers take their
+inputs from here, and nothing else is shared between the two sides.
+
+Workloads follow the KnapSpec setting (arXiv 2602.20217, "KnapSpec:
+Self-Speculative Decoding via Adaptive Layer Selection as a Knapsack Problem",
+§3.1/§3.3 on the Pith review page): every Attention and every MLP sublayer of a
+decoder is one knapsack item, Attention latency grows linearly with context and
+MLP latency is flat.  The trained Qwen3/Llama3 weights and the benchmark texts
+the paper uses are not available, so every tensor here is drawn at random:
+
+* linear weights ~ N(0, 0.02^2), stored as ``[out_features][in_features]``
+  (bf16, or fp32 for the tiny model); RMSNorm gains are ones;
+* the key/value cache ~ N(0, (0.02*sqrt(d_model))^2) per entry -- the per-entry
+  spread that projecting a unit-RMS hidden state through N(0, 0.02^2) weights
+  gives -- laid out ``[layer][position][kv_head][head_dim]``;
+* the T evaluation tokens' input hidden states x0 ~ N(0, 1), ``[T][d_model]`` fp32.
+
+Draw order (one ``torch.Generator`` seeded with ``seed`` on ``device``): for each
+layer in order Wq, Wo, W_gate, W_up, W_down; then the K cache, the V cache, then
+x0.  Each tensor is drawn in fp32 and then rounded to the storage dtype.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic decoder + DP problem."""
+
+    name: str
+    n_layers: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    rms_eps: float
+    rope_base: float
+    ctx: int                 # context tokens already in the cache
+    T: int                   # evaluation tokens (the DP's r / m window)
+    wdtype: str              # "f32" or "bf16" (weights and KV cache)
+    n_bins: int              # budget-grid bins used by the latency quantiser
+    gamma_max: int           # largest draft length in the TPT grid search
+    gen_device: str          # device whose RNG defines the values ("cpu"/"cuda")
+    contexts: Sequence[int] = ()   # extra contexts a re-solve sweep visits
+    attn_latency: str = "1+ctx/256"  # latency model (stated by the workload)
+    mlp_latency: float = 4.0
+
+    @property
+    def n_items(self) -> int:
+        return 2 * self.n_layers
+
+    @property
+    def q_dim(self) -> int:
+        return self.n_q_heads * self.head_dim
+
+    @property
+    def n_positions(self) -> int:
+        return self.ctx + self.T
+
+    def with_ctx(self, ctx: int) -> "Workload":
+        return dataclasses.replace(self, ctx=ctx)
+
+    def latencies(self, ctx: Optional[int] = None) -> List[float]:
+        """Raw per-item latencies t_i (item 2l = Attn of layer l, 2l+1 = MLP).
+
+        These are the workload's stated latency model (synthetic stand-ins for
+        the paper's pre-profiled hardware latencies): an Attention sublayer costs
+        an affine function of the context length, an MLP sublayer a constant.
+        """
+        c = self.ctx if ctx is None else ctx
+        if self.attn_latency == "2+ceil(ctx/64)":
+            ta = 2.0 + float(-(-c // 64))
+        elif self.attn_latency == "1+ctx/256":
+            ta = 1.0 + c / 256.0
+        else:
+            raise ValueError(self.attn_latency)
+        out: List[float] = []
+        for _ in range(self.n_layers):
+            out += [ta, float(self.mlp_latency)]
+        return out
+
+
+WORKLOADS: Dict[str, Workload] = {
+    # Tiny Llama-style decoder, fp32: small enough for exhaustive subset search.
+    "tiny": Workload("tiny", n_layers=4, d_model=256, n_q_heads=4, n_kv_heads=4,
+                     head_dim=64, ffn=688, rms_eps=1e-6, rope_base=1e4, ctx=128, T=4,
+                     wdtype="f32", n_bins=28, gamma_max=8, gen_device="cpu",
+                     attn_latency="2+ceil(ctx/64)", mlp_latency=3.0),
+    # Small GQA decoder, bf16.
+    "small": Workload("small", n_layers=16, d_model=1024, n_q_heads=16, n_kv_heads=4,
+                      head_dim=64, ffn=2816, rms_eps=1e-6, rope_base=1e4, ctx=2048, T=8,
+                      wdtype="bf16", n_bins=256, gamma_max=8, gen_device="cpu"),
+    # Llama-3-8B shape at 8k context.
+    "llama3_8b_8k": Workload("llama3_8b_8k", n_layers=32, d_model=4096, n_q_heads=32,
+                             n_kv_heads=8, head_dim=128, ffn=14336, rms_eps=1e-6,
+                             rope_base=5e5, ctx=8192, T=16, wdtype="bf16", n_bins=512,
+                             gamma_max=10, gen_device="cuda"),
+    # Llama-3-8B shape, long context, re-solved at 4k / 16k / 32k.
+    "llama3_8b_32k": Workload("llama3_8b_32k", n_layers=32, d_model=4096, n_q_heads=32,
+                              n_kv_heads=8, head_dim=128, ffn=14336, rms_eps=1e-6,
+                              rope_base=5e5, ctx=32768, T=16, wdtype="bf16", n_bins=1024,
+                              gamma_max=10, gen_device="cuda",
+                              contexts=(4096, 16384, 32768)),
+    # Qwen3-32B shape at 16k context (q-dim 8192 differs from d_model 5120).
+    "qwen3_32b_16k": Workload("qwen3_32b_16k", n_layers=64, d_model=5120, n_q_heads=64,
+                              n_kv_heads=8, head_dim=128, ffn=25600, rms_eps=1e-6,
+                              rope_base=1e6, ctx=16384, T=8, wdtype="bf16", n_bins=1024,
+                              gamma_max=10, gen_device="cuda"),
+}
+
+# Order of the five workloads as the build's configuration list names them.
+WORKLOAD_ORDER = ["tiny", "small", "llama3_8b_8k", "llama3_8b_32k", "qwen3_32b_16k"]
+
+LINEAR_STD = 0.02
+
+
+def kv_std(wl: Workload) -> float:
+    """Per-entry standard deviation of the synthetic K/V cache."""
+    return LINEAR_STD * math.sqrt(wl.d_model)
+
+
+def torch_dtype(wl: Workload) -> torch.dtype:
+    return torch.float32 if wl.wdtype == "f32" else torch.bfloat16
+
+
+@dataclasses.dataclass
+class Inputs:
+    """Seeded inputs of one workload, all on one device."""
+
+    wl: Workload
+    layers: List[Dict[str, torch.Tensor]]   # per layer: attn_norm, wq, wo, mlp_norm, w_gate, w_up, w_down
+    k_cache: torch.Tensor                    # [L][ctx+T][Hkv][hd]
+    v_cache: torch.Tensor                    # [L][ctx+T][Hkv][hd]
+    x0: torch.Tensor                         # [T][d] fp32
+
+    def first_layers(self, n: int) -> "Inputs":
+        """The sub-problem made of the first ``n`` layers (same cache rows and x0)."""
+        return Inputs(dataclasses.replace(self.wl, n_layers=n), self.layers[:n],
+                      self.k_cache[:n], self.v_cache[:n], self.x0)
+
+    def to(self, device) -> "Inputs":
+        mv = lambda t: t.to(device)
+        return Inputs(self.wl, [{k: mv(v) for k, v in l.items()} for l in self.layers],
+                      mv(self.k_cache), mv(self.v_cache), mv(self.x0))
+
+
+def _randn(shape, std, dtype, gen, device):
+    t = torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def make_inputs(wl: Workload, seed: int = 0, device: Optional[str] = None) -> Inputs:
+    """Draw the workload's inputs (see the module docstring for the recipe)."""
+    dev = device or wl.gen_device
+    if dev == "cuda" and not torch.cuda.is_available():
+        raise RuntimeError(f"workload {wl.name} is drawn on CUDA, which is not available")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dt = torch_dtype(wl)
+    L = wl.n_layers
+    d, qd, F = wl.d_model, wl.q_dim, wl.ffn
+    layers = []
+    for _ in range(L):
+        layer = {
+            "wq": _randn((qd, d), LINEAR_STD, dt, gen, dev),
+            "wo": _randn((d, qd), LINEAR_STD, dt, gen, dev),
+            "w_gate": _randn((F, d), LINEAR_STD, dt, gen, dev),
+            "w_up": _randn((F, d), LINEAR_STD, dt, gen, dev),
+            "w_down": _randn((d, F), LINEAR_STD, dt, gen, dev),
+        }
+        layer["attn_norm"] = torch.ones(d, dtype=dt, device=dev)
+        layer["mlp_norm"] = torch.ones(d, dtype=dt, device=dev)
+        layers.append(layer)
+    kvshape = (L, wl.n_positions, wl.n_kv_heads, wl.head_dim)
+    k_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
+    v_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
+    x0 = _randn((wl.T, d), 1.0, torch.float32, gen, dev)
+    return Inputs(wl, layers, k_cache, v_cache, x0)
+
+
+def truncated(wl: Workload, n_layers: int, ctx: Optional[int] = None) -> Workload:
+    """The same workload shape with fewer layers (and optionally another context)."""
+    return dataclasses.replace(wl, n_layers=n_layers, ctx=wl.ctx if ctx is None else ctx)
+
+
+def random_states(shape: Sequence[int], seed: int, device: str = "cpu",
+                  dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """N(0,1) tensor of the given shape (for kernel-level tests of one step)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32).to(dtype)
