@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark of the KnapSpec DP solve (the whole hot path: reference states,
+batched sublayer forwards over every budget cell, select/backpointer,
+reconstruction and the TPT search) on the synthetic Llama-3-8B-shaped workload.
+
+One step = one ks_solve over inputs already resident in HBM.  Prints one JSON
+line.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded
+sample of the same workload.  Under torchrun every rank solves its own
+independent replica (the DP has no data-path exchange), and the reported time
+is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from knapsack_layer_selection_b200 import workloads as W  # noqa: E402
+
+METRIC = "KnapSpec DP solve ms & budget-cell·sublayer/s (8B shape), % of roofline"
+UNIT = "budget-cell·sublayer/s"
+DEFAULT_WORKLOAD = "llama3_8b_8k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TENSOR_KINDS = ("gemm_q_rope", "gemm_o_residual", "gemm_gateup_swiglu", "gemm_down_residual",
+                "attention")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="CPU work the oracle baseline sample aims for")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="ks_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- workload helpers
+def solver_for(wl, inp, keep=False):
+    from knapsack_layer_selection_b200 import binding as B
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    prm = B.params(wl.gamma_max, wl.n_bins)
+    return B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, wl.latencies(), prm,
+                    keep_bp=keep, keep_cos=False, keep_tpt=keep, keep_ref=keep)
+
+
+def oracle_sample(wl, inp, seconds: float):
+    """Time the oracle (as it stands) on a bounded sample of the workload.
+
+    Sample: the DP over the first layer's two items and the lowest n_cells
+    budgets (plus that layer's reference states), repeated until `seconds` of
+    CPU work.  Returns (cells*items per second, description, threads used).
+    """
+    from oracle import ks_oracle as O
+    layer = {k: v.detach().float().cpu().numpy() for k, v in inp.layers[0].items()}
+    kc = [inp.k_cache[0].detach().float().cpu().numpy()]
+    vc = [inp.v_cache[0].detach().float().cpu().numpy()]
+    m = O.Model(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rms_eps, wl.rope_base, [layer], kc, vc)
+    x0 = inp.x0.detach().double().cpu().numpy()
+    t = wl.latencies()[:2]
+    w = O.quantize_weights(wl.latencies(), wl.n_bins)[:2]
+    n_cells = max(w) + 16
+    runs, elapsed = 0, 0.0
+    while runs == 0 or elapsed < seconds:
+        t0 = time.perf_counter()
+        O.dp_solve(m, x0, wl.ctx, w, t, wl.gamma_max, n_cells=n_cells)
+        elapsed += time.perf_counter() - t0
+        runs += 1
+    units = n_cells * 2 * runs
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    desc = (f"{wl.name}: DP over layer 0's Attn+MLP items and budgets 0..{n_cells - 1} "
+            f"({n_cells} cells x 2 items, incl. that layer's reference states), {runs} run(s)")
+    return units / elapsed, desc, threads, elapsed / runs
+
+
+def base_config(wl, C, world):
+    return {"workload": wl.name, "budget_cells": C, "items": wl.n_items, "T": wl.T,
+            "ctx": wl.ctx, "d_model": wl.d_model, "ffn": wl.ffn,
+            "l2": "inputs larger than L2: every solve streams all weights "
+                  f"({wl.n_layers} layers) and the KV cache from HBM",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
+# ---------------------------------------------------------------- the reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(wl, device=dev if wl.gen_device == "cuda" else "cpu")
+    from oracle import ks_oracle as O
+    C = sum(O.quantize_weights(wl.latencies(), wl.n_bins)) + 1
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wl, inp, 0.0)
+    vals, secs, desc, threads = [], [], "", 1
+    for _ in range(args.steps):
+        v, desc, threads, s = oracle_sample(wl, inp, per_step)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * statistics.mean(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": base_config(wl, C, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    from knapsack_layer_selection_b200 import binding as B
+    from knapsack_layer_selection_b200 import build as BUILD
+    if rank == 0:
+        BUILD.build()
+    barrier(world)
+    wl = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(wl, seed=rank, device="cuda")
+    solver = solver_for(wl, inp)
+    C = solver.C
+    units = C * wl.n_items                     # budget-cell x sublayer evaluations per solve
+    x0 = inp.x0
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(3, args.warmup)):
+        solver.solve(x0)
+    torch.cuda.synchronize()
+    solver.check_status()
+
+    # ---- device-timed region
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        B.profile_start(timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            solver.solve(x0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        stats = B.profile_stop()
+    barrier(world)
+    solver.check_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world)
+    value = world * units / (ms / 1000.0)
+
+    # ---- end to end through the public API with host buffers
+    words = (wl.n_items + 63) // 64
+    x0_host = x0.detach().cpu().pin_memory()
+    x0_dev = torch.empty_like(x0)
+    vals_h = torch.empty(C, dtype=torch.float32).pin_memory()
+    sets_h = torch.empty(C, words, dtype=torch.int64).pin_memory()
+    best_h = torch.empty(2, dtype=torch.int32).pin_memory()
+    h2d = x0_host.numel() * 4
+    d2h = vals_h.numel() * 4 + sets_h.numel() * 8 + best_h.numel() * 4
+    barrier(world)
+    torch.cuda.synchronize()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        x0_dev.copy_(x0_host, non_blocking=True)
+        out = solver.solve(x0_dev)
+        vals_h.copy_(out.values, non_blocking=True)
+        sets_h.copy_(out.sets, non_blocking=True)
+        best_h.copy_(out.best, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3) / args.steps, world)
+
+    # ---- roofline of the dominant kernel (live event times)
+    peaks, peak_src = load_peaks()
+    kinds = {s["name"]: s for s in stats}
+    dom = max(stats, key=lambda s: s["total_ms"])
+    per_launch_ms = dom["total_ms"] / max(1, dom["launches"])
+    if dom["name"] in TENSOR_KINDS:
+        achieved = dom["flops"] / (dom["total_ms"] / 1000.0) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        roof = {"bound": "tensor", "unit": "TFLOP/s"}
+    else:
+        achieved = dom["bytes"] / (dom["total_ms"] / 1000.0) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s"}
+    roof.update({"kernel": dom["name"], "achieved": achieved, "peak": peak,
+                 "frac": achieved / peak, "traffic": None,
+                 "peak_source": f"{peak_src} (sustained bf16)" if roof["bound"] == "tensor"
+                 else f"{peak_src} hbm copy",
+                 "launches": dom["launches"] // args.steps, "ms_per_launch": per_launch_ms})
+    flops = sum(s["flops"] for s in stats if s["name"] in TENSOR_KINDS) / args.steps
+    weight_bytes = sum(p.numel() * p.element_size() for l in inp.layers for p in l.values())
+    kv_bytes = 2 * wl.n_layers * (wl.ctx + wl.T) * wl.n_kv_heads * wl.head_dim * 2
+    t_flop = flops / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12)
+    t_bytes = (weight_bytes + kv_bytes) / (peaks["hbm_gbs"] * 1e9)
+    solve_roof_ms = 1000.0 * max(t_flop, t_bytes)
+    launches = sum(s["launches"] for s in stats) // args.steps
+
+    cpu = None
+    if rank == 0 and world == 1:
+        v, desc, threads, _ = oracle_sample(wl, inp, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        cfg = base_config(wl, C, world)
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if wl.wdtype == "bf16" else "f32", "data": "synthetic",
+                "config": cfg,
+                "solve_ms": ms,
+                "solve_roofline": {"ms": solve_roof_ms, "frac": solve_roof_ms / ms,
+                                   "tensor_flops": flops, "weight_kv_bytes": weight_bytes + kv_bytes,
+                                   "peak_source": peak_src},
+                "roofline": roof,
+                "cpu_baseline": cpu,
+                "e2e": {"value": world * units / (e2e_ms / 1000.0), "unit": UNIT,
+                        "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches * args.steps,
+                "kernels": {s["name"]: {"launches_per_step": s["launches"] // args.steps,
+                                        "ms_per_step": s["total_ms"] / args.steps,
+                                        "share": s["total_ms"] / max(1e-9, sum(x["total_ms"] for x in stats))}
+                            for s in stats},
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,276 @@
+/*
+ * knapspec.h -- C ABI of the B200 (sm_100a) KnapSpec knapsack layer-selection DP.
+ *
+ * Method: "KnapSpec: Self-Speculative Decoding via Adaptive Layer Selection as a
+ * Knapsack Problem" (arXiv 2602.20217), as the Pith review page of the paper
+ * describes it.  Every Attention and every MLP sublayer of a decoder is one
+ * knapsack item whose integer weight is its latency (review, "What carries the
+ * argument"; referee major 4 on §3.6).  For every latency-budget cell b the DP
+ * keeps whichever of "skip item i" (carry cell b) and "execute item i" (run the
+ * sublayer on cell b - w_i) has the higher cosine similarity to the full
+ * model's hidden state X^(i) (Eq. 6-8, Algorithm 1; referee major 1), stores a
+ * backpointer, reads one layer set per budget back (Algorithm 2; referee minor
+ * 4) and grid-searches the draft length gamma for the largest Tokens-per-Time
+ * TPT(S, gamma) = ((1 - a^(gamma+1)) / (1 - a)) / (gamma t_Draft(S) + t_Target)
+ * (Eq. 4, Eq. 5).
+ *
+ * Conventions shared by every call:
+ *  - Items are numbered k = 0 .. 2L-1: item 2l is the Attention sublayer of
+ *    layer l, item 2l+1 its MLP sublayer.  X^(0) is the T evaluation tokens'
+ *    input state, X^(k+1) = item_k(X^(k)).
+ *  - Budget cells b = 0 .. C-1 with C = K + 1 and K = sum of the item weights.
+ *    A cell holds the best state that uses at most b weight units; every cell
+ *    starts from X^(0).  Execute reads cell b - w_k and wins only when its
+ *    value is strictly larger.
+ *  - The value of a state H [T][d] is the mean over tokens of the per-token
+ *    cosine with the target state.
+ *  - Pointers named "device" are CUDA device pointers (cudaMalloc or a
+ *    torch CUDA tensor); "host" pointers are ordinary host memory.  The caller
+ *    owns every buffer; the library allocates nothing.  All dense arrays are
+ *    row-major and contiguous.
+ *  - Calls that take a stream are asynchronous on it: they validate their
+ *    arguments on the host, enqueue kernels and return.  Results are valid
+ *    once the stream has been synchronised.  Host-side argument errors return
+ *    a ks_status before anything is enqueued; the text is in ks_last_error().
+ *    A kernel that gives up a bounded wait writes KS_ERR_TIMEOUT into the
+ *    caller's device status word (ks_result.status) and returns; kernels never
+ *    trap.
+ *  - Linear weights are stored [out_features][in_features] (the layout of
+ *    torch.nn.Linear.weight).  Weights and the KV cache are bf16 (KS_BF16) or
+ *    fp32 (KS_F32); hidden states are always fp32.
+ */
+#ifndef KNAPSPEC_H
+#define KNAPSPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KS_API __attribute__((visibility("default")))
+#else
+#define KS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef void* ks_stream_t;
+
+typedef enum {
+  KS_OK = 0,
+  KS_ERR_INVALID_ARG = 1,   /* bad pointer, size or shape */
+  KS_ERR_UNSUPPORTED = 2,   /* shape or dtype the kernels do not handle */
+  KS_ERR_WORKSPACE = 3,     /* workspace smaller than ks_workspace_size() */
+  KS_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+  KS_ERR_TIMEOUT = 5,       /* device side: a bounded wait expired */
+  KS_ERR_INTERNAL = 6
+} ks_status;
+
+typedef enum { KS_F32 = 0, KS_BF16 = 1 } ks_dtype;
+
+/* Decoder shape.  head_dim must be 64 or 128; n_q_heads a multiple of
+ * n_kv_heads; d_model a multiple of 64; ffn a multiple of 16. */
+typedef struct {
+  int32_t n_layers;
+  int32_t d_model;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t ffn;
+  float rms_eps;       /* RMSNorm: x / sqrt(mean(x^2) + eps) * gain */
+  double rope_base;    /* rotate-half RoPE, theta_j = base^(-2j/head_dim) */
+  int32_t wdtype;      /* ks_dtype of the weights and the KV cache */
+} ks_model_desc;
+
+/* Device pointers to one layer's weights (dtype = ks_model_desc.wdtype):
+ * attn_norm [d], wq [Hq*hd][d], wo [d][Hq*hd], mlp_norm [d],
+ * w_gate [ffn][d], w_up [ffn][d], w_down [d][ffn].
+ * Wk/Wv are not needed: the DP reads keys and values from the cache. */
+typedef struct {
+  const void* attn_norm;
+  const void* wq;
+  const void* wo;
+  const void* mlp_norm;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+} ks_layer_weights;
+
+/* The full model's KV cache (device, dtype = wdtype), laid out
+ * [n_layers][cache_rows][n_kv_heads][head_dim] for K and for V, keys already
+ * rotated.  Evaluation token t (0 .. T-1) sits at position ctx + t and attends
+ * to positions 0 .. ctx + t, so cache_rows >= ctx + T. */
+typedef struct {
+  const void* k_cache;
+  const void* v_cache;
+  int64_t cache_rows;
+  int32_t ctx;
+} ks_cache_desc;
+
+/* Selection parameters.  alpha(b) = clamp((value_b - alpha_lo) / alpha_scale,
+ * 0, alpha_max) is the acceptance-rate stand-in; gamma runs 1 .. gamma_max. */
+typedef struct {
+  int32_t gamma_max;
+  int32_t n_bins;      /* budget-grid bins for ks_quantize_weights (ks_solve
+                          uses it when no weights are passed) */
+  double alpha_lo;
+  double alpha_scale;
+  double alpha_max;
+} ks_params;
+
+/* Outputs of ks_solve: caller-allocated DEVICE buffers.  C = K + 1 cells,
+ * words = ceil(n_items / 64).  Optional buffers may be NULL. */
+typedef struct {
+  int32_t* status;     /* [1] required: 0, or a ks_status a kernel wrote */
+  float* values;       /* [C] required: final-row value of every cell */
+  uint64_t* sets;      /* [C][words] required: bit k set = item k executed */
+  int32_t* used_w;     /* [C] optional: sum of the executed items' weights */
+  double* t_draft;     /* [C] optional: sum of the executed items' latencies */
+  uint8_t* bp;         /* [n_items][C] optional: 1 = execute won */
+  float* cos_skip;     /* [n_items][C] optional: skip candidate's value */
+  float* cos_exec;     /* [n_items][C] optional: execute candidate's value (NaN if b < w) */
+  double* tpt;         /* [C][gamma_max] optional: the TPT grid */
+  int32_t* best;       /* [2] required: best cell b*, best gamma* */
+  double* best_tpt;    /* [1] optional: TPT(b*, gamma*) */
+  float* ref_states;   /* [n_items+1][T][d] optional: the reference states used */
+} ks_result;
+
+/* Library version string (static storage). */
+KS_API const char* ks_version(void);
+
+/* Text of the last host-side error of the calling thread ("" if none). */
+KS_API const char* ks_last_error(void);
+
+/* Static text naming a status code. */
+KS_API const char* ks_status_string(ks_status s);
+
+/*
+ * a0 -- latency weights (review, referee major 4 on §3.6: w_Attn ~ t_Attn/Delta).
+ * Host only.  t: host [n_items] positive latencies; w_out: host [n_items].
+ * Delta = sum(t) / n_bins (summed in item order), w_k = max(1, floor(t_k/Delta + 1/2)).
+ * Errors: KS_ERR_INVALID_ARG for NULL pointers, n_items < 1, n_bins < 1 or a
+ * latency that is not positive.
+ */
+KS_API ks_status ks_quantize_weights(const double* t, int32_t n_items, int32_t n_bins, int32_t* w_out);
+
+/*
+ * Workspace bytes ks_solve / ks_reference_forward / ks_sublayer_forward need
+ * for a model, a batch of up to n_cells budget cells and T evaluation tokens.
+ * Host only.  The workspace is a caller-owned device buffer, 256-byte aligned,
+ * used as scratch; one workspace must not be shared by calls that overlap.
+ */
+KS_API ks_status ks_workspace_size(const ks_model_desc* model, int32_t n_cells, int32_t T, size_t* bytes);
+
+/*
+ * a2 / a3 -- one sublayer on a batch of E states (Eq. 7's "execute" branch).
+ * Attention (item 2l): H + Wo . Attn(RoPE(Wq . RMSNorm(H))) with causal GQA
+ * over the cache; MLP (item 2l+1): H + W_down (silu(W_gate x) * W_up x),
+ * x = RMSNorm(H).
+ * states_in, states_out: device [E][T][d] fp32 (must not overlap).
+ * Errors: KS_ERR_INVALID_ARG / KS_ERR_UNSUPPORTED / KS_ERR_WORKSPACE on the host.
+ */
+KS_API ks_status ks_sublayer_forward(const ks_model_desc* model, const ks_layer_weights* layers,
+                              const ks_cache_desc* cache, int32_t T, int32_t item,
+                              const float* states_in, int32_t E, float* states_out,
+                              void* workspace, size_t workspace_bytes, ks_stream_t stream);
+
+/*
+ * a1 -- the full model's reference states (the X^(i) of Eq. 6/7):
+ * ref_out[0] = x0, ref_out[k+1] = item_k(ref_out[k]).
+ * layers: HOST array [n_layers] of device weight pointers.  x0: device [T][d]
+ * fp32.  ref_out: device [n_items+1][T][d] fp32.
+ */
+KS_API ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer_weights* layers,
+                               const ks_cache_desc* cache, int32_t T, const float* x0,
+                               float* ref_out, void* workspace, size_t workspace_bytes,
+                               ks_stream_t stream);
+
+/*
+ * a4 -- one DP row's select step (Eq. 7/8): for every cell b in 0 .. C-1,
+ *   s = meancos(prev[b], target), e = meancos(exec[b - w], target) if b >= w,
+ *   cur[b] = exec[b - w] if e > s else prev[b];  val[b], bp[b] record the choice.
+ * prev, cur: device [C][T][d] fp32 (must not overlap); exec: device [C-w][T][d]
+ * fp32 (exec[e] belongs to cell e + w); target: device [T][d] fp32.
+ * val: device [C] fp32; bp: device [C] u8; cos_skip / cos_exec: device [C] fp32
+ * or NULL.  Cosines are accumulated in fp64.  w >= 1.
+ */
+KS_API ks_status ks_select_step(const float* prev, const float* exec, const float* target,
+                         int32_t C, int32_t T, int32_t d, int32_t w, float* cur, float* val,
+                         uint8_t* bp, float* cos_skip, float* cos_exec, ks_stream_t stream);
+
+/*
+ * a5 -- set reconstruction (Algorithm 2 with stored backpointers): for every
+ * cell b, walk j = b from the last item down; item k is in the set when
+ * bp[k][j] = 1, and then j -= w[k].
+ * bp: device [n_items][C] u8; w: device [n_items] int32; t: device [n_items]
+ * fp64.  sets: device [C][words]; used_w: device [C] int32 (or NULL); t_draft:
+ * device [C] fp64 (or NULL), summed over the set in increasing item order.
+ * A walk that would leave the grid writes KS_ERR_INTERNAL to status (device [1]).
+ */
+KS_API ks_status ks_reconstruct(const uint8_t* bp, const int32_t* w, const double* t, int32_t n_items,
+                         int32_t C, uint64_t* sets, int32_t* used_w, double* t_draft,
+                         int32_t* status, ks_stream_t stream);
+
+/*
+ * a6 -- TPT grid search (Eq. 4, Eq. 5) in fp64: for every cell b and gamma in
+ * 1 .. gamma_max, TPT = (sum_{k=0..gamma} a_b^k) / (gamma t_draft[b] + t_target)
+ * with a_b = clamp((values[b] - alpha_lo)/alpha_scale, 0, alpha_max); the
+ * geometric sum is taken term by term.  The best pair is the largest TPT, ties
+ * to the smaller b, then the smaller gamma.
+ * values: device [C] fp32; t_draft: device [C] fp64; tpt: device
+ * [C][gamma_max] fp64 or NULL; best: device [2] int32 (b*, gamma*);
+ * best_tpt: device [1] fp64 or NULL.
+ */
+KS_API ks_status ks_tpt_argmax(const float* values, const double* t_draft, int32_t C, double t_target,
+                        const ks_params* params, double* tpt, int32_t* best, double* best_tpt,
+                        ks_stream_t stream);
+
+/*
+ * a0-a6 -- the whole DP on one GPU (the spec call).
+ * layers: HOST array [n_layers] of device weight pointers; cache: the full
+ * model's KV cache; x0: device [T][d] fp32; ref: device [n_items+1][T][d] fp32
+ * reference states, or NULL to compute them with ks_reference_forward's
+ * kernels; w: HOST [n_items] item weights, or NULL to quantise t with
+ * params->n_bins; t: HOST [n_items] latencies (t_Target = their sum).
+ * The number of cells is C = sum(w) + 1; out's buffers must be sized for it
+ * (ks_solve_cells() returns C).  The workspace must hold
+ * ks_workspace_size(model, C, T).  Nothing is copied back to the host.
+ */
+KS_API ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
+                   const ks_cache_desc* cache, int32_t T, const float* x0, const float* ref,
+                   const int32_t* w, const double* t, const ks_params* params,
+                   void* workspace, size_t workspace_bytes, ks_result* out, ks_stream_t stream);
+
+/* C = sum(w) + 1 for the weights ks_solve would use (w, or t quantised with
+ * params->n_bins when w is NULL).  Host only. */
+KS_API ks_status ks_solve_cells(int32_t n_items, const int32_t* w, const double* t,
+                         const ks_params* params, int32_t* n_cells);
+
+/*
+ * Launch accounting.  Between ks_profile_start and ks_profile_stop the library
+ * counts the kernels it enqueues per kind, adds up their algorithmic FLOPs and
+ * bytes (the work the DP defines, not what the hardware moved) and, when
+ * timing != 0, records a CUDA event pair on the launching stream around each
+ * kind's launches (not while the stream is being captured into a graph).
+ * ks_profile_stop waits for those events, fills up to `capacity` entries (one
+ * per kind that launched) and reports the number of kinds in *n_kinds.
+ * Process-wide state; calls from several threads are serialised.
+ */
+typedef struct {
+  char name[32];
+  int64_t launches;
+  double total_ms;     /* summed event time (0 when timing was off) */
+  double flops;        /* algorithmic floating-point operations */
+  double bytes;        /* algorithmic HBM bytes */
+} ks_kernel_stat;
+
+KS_API ks_status ks_profile_start(int32_t timing);
+KS_API ks_status ks_profile_stop(ks_kernel_stat* stats, int32_t capacity, int32_t* n_kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KNAPSPEC_H */

@@ -1,0 +1,334 @@
+"""Thin ctypes binding of libknapspec.so (include/knapspec.h).
+
+Every function here only marshals arguments: it checks tensor devices, dtypes
+and shapes, turns them into pointers and calls the C ABI on the current torch
+CUDA stream.  All arithmetic of the DP runs in the library's CUDA kernels.  If
+the library has not been built the first call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libknapspec.so")
+
+KS_F32, KS_BF16 = 0, 1
+
+
+class KnapSpecError(RuntimeError):
+    pass
+
+
+class ModelDesc(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("rms_eps", ctypes.c_float), ("rope_base", ctypes.c_double),
+                ("wdtype", ctypes.c_int32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down")]
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("cache_rows", ctypes.c_int64), ("ctx", ctypes.c_int32)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("gamma_max", ctypes.c_int32), ("n_bins", ctypes.c_int32),
+                ("alpha_lo", ctypes.c_double), ("alpha_scale", ctypes.c_double),
+                ("alpha_max", ctypes.c_double)]
+
+
+class Result(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("status", "values", "sets", "used_w", "t_draft", "bp", "cos_skip",
+                 "cos_exec", "tpt", "best", "best_tpt", "ref_states")]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weights",
+           "ks_workspace_size", "ks_sublayer_forward", "ks_reference_forward",
+           "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
+           "ks_profile_start", "ks_profile_stop"]
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libknapspec.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise KnapSpecError(f"{LIB_PATH} is missing: build it with "
+                            "`python -m knapsack_layer_selection_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, D, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+    sig = {
+        "ks_version": ([], ctypes.c_char_p),
+        "ks_last_error": ([], ctypes.c_char_p),
+        "ks_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "ks_quantize_weights": ([P, I32, I32, P], ctypes.c_int),
+        "ks_workspace_size": ([P, I32, I32, ctypes.POINTER(SZ)], ctypes.c_int),
+        "ks_sublayer_forward": ([P, P, P, I32, I32, P, I32, P, P, SZ, P], ctypes.c_int),
+        "ks_reference_forward": ([P, P, P, I32, P, P, P, SZ, P], ctypes.c_int),
+        "ks_select_step": ([P, P, P, I32, I32, I32, I32, P, P, P, P, P, P], ctypes.c_int),
+        "ks_reconstruct": ([P, P, P, I32, I32, P, P, P, P, P], ctypes.c_int),
+        "ks_tpt_argmax": ([P, P, I32, D, P, P, P, P, P], ctypes.c_int),
+        "ks_solve": ([P, P, P, I32, P, P, P, P, P, P, SZ, P, P], ctypes.c_int),
+        "ks_solve_cells": ([I32, P, P, P, ctypes.POINTER(I32)], ctypes.c_int),
+        "ks_profile_start": ([I32], ctypes.c_int),
+        "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        lib = load()
+        raise KnapSpecError(f"{lib.ks_status_string(status).decode()}: "
+                            f"{lib.ks_last_error().decode()}")
+
+
+def _dev(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise KnapSpecError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise KnapSpecError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise KnapSpecError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def version() -> str:
+    return load().ks_version().decode()
+
+
+# ---------------------------------------------------------------- descriptors
+def model_desc(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, ffn, rms_eps, rope_base,
+               wdtype: str) -> ModelDesc:
+    return ModelDesc(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, ffn, rms_eps,
+                     rope_base, KS_F32 if wdtype == "f32" else KS_BF16)
+
+
+def layer_array(layers: Sequence[Dict[str, torch.Tensor]], wdtype: torch.dtype):
+    arr = (LayerWeights * len(layers))()
+    for i, L in enumerate(layers):
+        for name in ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down"):
+            setattr(arr[i], name, _dev(L[name], wdtype, f"layers[{i}].{name}"))
+    return arr
+
+
+def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int) -> CacheDesc:
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
+        raise KnapSpecError("k_cache / v_cache must both be [L][rows][Hkv][hd]")
+    return CacheDesc(_dev(k_cache, name="k_cache"), _dev(v_cache, name="v_cache"),
+                     k_cache.shape[1], ctx)
+
+
+def params(gamma_max: int, n_bins: int = 0, alpha_lo: float = 0.5, alpha_scale: float = 0.5,
+           alpha_max: float = 0.99) -> Params:
+    return Params(gamma_max, n_bins, alpha_lo, alpha_scale, alpha_max)
+
+
+# ---------------------------------------------------------------- calls
+def quantize_weights(t: Sequence[float], n_bins: int) -> List[int]:
+    n = len(t)
+    tt = (ctypes.c_double * n)(*t)
+    w = (ctypes.c_int32 * n)()
+    _check(load().ks_quantize_weights(tt, n, n_bins, w))
+    return list(w)
+
+
+def workspace_size(model: ModelDesc, n_cells: int, T: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load().ks_workspace_size(ctypes.byref(model), n_cells, T, ctypes.byref(out)))
+    return out.value
+
+
+def workspace(model: ModelDesc, n_cells: int, T: int, device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(model, n_cells, T), dtype=torch.uint8, device=device)
+
+
+def sublayer_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, item: int,
+                     states_in: torch.Tensor, states_out: torch.Tensor,
+                     ws: torch.Tensor) -> None:
+    E = states_in.shape[0] if states_in.dim() == 3 else 1
+    _check(load().ks_sublayer_forward(ctypes.byref(model), layers, ctypes.byref(cache), T, item,
+                                      _dev(states_in, torch.float32, "states_in"), E,
+                                      _dev(states_out, torch.float32, "states_out"),
+                                      _dev(ws, name="workspace"), ws.numel(), _stream()))
+
+
+def reference_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, x0: torch.Tensor,
+                      ref_out: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(load().ks_reference_forward(ctypes.byref(model), layers, ctypes.byref(cache), T,
+                                       _dev(x0, torch.float32, "x0"),
+                                       _dev(ref_out, torch.float32, "ref_out"),
+                                       _dev(ws, name="workspace"), ws.numel(), _stream()))
+
+
+def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:
+    C, T, d = prev.shape
+    _check(load().ks_select_step(_dev(prev, torch.float32, "prev"),
+                                 _dev(exec_, torch.float32, "exec"),
+                                 _dev(target, torch.float32, "target"), C, T, d, w,
+                                 _dev(cur, torch.float32, "cur"), _dev(val, torch.float32, "val"),
+                                 _dev(bp, torch.uint8, "bp"),
+                                 _dev(cos_skip, torch.float32, "cos_skip"),
+                                 _dev(cos_exec, torch.float32, "cos_exec"), _stream()))
+
+
+def reconstruct(bp: torch.Tensor, w: torch.Tensor, t: torch.Tensor, sets: torch.Tensor,
+                used_w: Optional[torch.Tensor], t_draft: Optional[torch.Tensor],
+                status: torch.Tensor) -> None:
+    n_items, C = bp.shape
+    _check(load().ks_reconstruct(_dev(bp, torch.uint8, "bp"), _dev(w, torch.int32, "w"),
+                                 _dev(t, torch.float64, "t"), n_items, C,
+                                 _dev(sets, torch.int64, "sets"),
+                                 _dev(used_w, torch.int32, "used_w"),
+                                 _dev(t_draft, torch.float64, "t_draft"),
+                                 _dev(status, torch.int32, "status"), _stream()))
+
+
+def tpt_argmax(values: torch.Tensor, t_draft: torch.Tensor, t_target: float, prm: Params,
+               tpt: Optional[torch.Tensor], best: torch.Tensor,
+               best_tpt: Optional[torch.Tensor]) -> None:
+    _check(load().ks_tpt_argmax(_dev(values, torch.float32, "values"),
+                                _dev(t_draft, torch.float64, "t_draft"), values.numel(),
+                                t_target, ctypes.byref(prm), _dev(tpt, torch.float64, "tpt"),
+                                _dev(best, torch.int32, "best"),
+                                _dev(best_tpt, torch.float64, "best_tpt"), _stream()))
+
+
+def solve_cells(t: Sequence[float], prm: Params, w: Optional[Sequence[int]] = None) -> int:
+    n = len(t)
+    tt = (ctypes.c_double * n)(*t)
+    ww = (ctypes.c_int32 * n)(*w) if w is not None else None
+    out = ctypes.c_int32()
+    _check(load().ks_solve_cells(n, ww, tt, ctypes.byref(prm), ctypes.byref(out)))
+    return out.value
+
+
+@dataclass
+class SolveOutputs:
+    status: torch.Tensor
+    values: torch.Tensor
+    sets: torch.Tensor
+    used_w: torch.Tensor
+    t_draft: torch.Tensor
+    best: torch.Tensor
+    best_tpt: torch.Tensor
+    bp: Optional[torch.Tensor] = None
+    cos_skip: Optional[torch.Tensor] = None
+    cos_exec: Optional[torch.Tensor] = None
+    tpt: Optional[torch.Tensor] = None
+    ref_states: Optional[torch.Tensor] = None
+
+
+class Solver:
+    """Owns the device workspace and result buffers for repeated ks_solve calls."""
+
+    def __init__(self, model: ModelDesc, layers: Sequence[Dict[str, torch.Tensor]],
+                 k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int, T: int,
+                 t: Sequence[float], prm: Params, w: Optional[Sequence[int]] = None,
+                 keep_bp: bool = True, keep_cos: bool = False, keep_tpt: bool = True,
+                 keep_ref: bool = True, device="cuda"):
+        self.model = model
+        self.wdtype = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
+        self._layers_keep = layers
+        self.layers = layer_array(layers, self.wdtype)
+        self._cache_keep = (k_cache, v_cache)
+        self.cache = cache_desc(k_cache, v_cache, ctx)
+        self.T = T
+        self.t = list(map(float, t))
+        self.prm = prm
+        self.n_items = 2 * model.n_layers
+        if len(self.t) != self.n_items:
+            raise KnapSpecError("need one latency per item")
+        self.w = list(w) if w is not None else quantize_weights(self.t, prm.n_bins)
+        self.C = solve_cells(self.t, prm, self.w)
+        self.ws = workspace(model, self.C, T, device)
+        C, n, words = self.C, self.n_items, (self.n_items + 63) // 64
+        z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=device)
+        self.out = SolveOutputs(
+            status=z(1, dt=torch.int32), values=z(C, dt=torch.float32),
+            sets=z(C, words, dt=torch.int64), used_w=z(C, dt=torch.int32),
+            t_draft=z(C, dt=torch.float64), best=z(2, dt=torch.int32),
+            best_tpt=z(1, dt=torch.float64),
+            bp=z(n, C, dt=torch.uint8) if keep_bp else None,
+            cos_skip=z(n, C, dt=torch.float32) if keep_cos else None,
+            cos_exec=z(n, C, dt=torch.float32) if keep_cos else None,
+            tpt=z(C, prm.gamma_max, dt=torch.float64) if keep_tpt else None,
+            ref_states=z(n + 1, T, model.d_model, dt=torch.float32) if keep_ref else None)
+        o = self.out
+        p = lambda x: None if x is None else x.data_ptr()
+        self.result = Result(p(o.status), p(o.values), p(o.sets), p(o.used_w), p(o.t_draft),
+                             p(o.bp), p(o.cos_skip), p(o.cos_exec), p(o.tpt), p(o.best),
+                             p(o.best_tpt), p(o.ref_states))
+        self._t_arr = (ctypes.c_double * n)(*self.t)
+        self._w_arr = (ctypes.c_int32 * n)(*self.w)
+
+    def solve(self, x0: torch.Tensor, ref: Optional[torch.Tensor] = None) -> SolveOutputs:
+        """Enqueue one solve on the current stream (results valid after a sync)."""
+        _check(load().ks_solve(ctypes.byref(self.model), self.layers, ctypes.byref(self.cache),
+                               self.T, _dev(x0, torch.float32, "x0"),
+                               _dev(ref, torch.float32, "ref"), self._w_arr, self._t_arr,
+                               ctypes.byref(self.prm), _dev(self.ws), self.ws.numel(),
+                               ctypes.byref(self.result), _stream()))
+        return self.out
+
+    def check_status(self) -> None:
+        s = int(self.out.status.item())
+        if s != 0:
+            raise KnapSpecError(f"device status {s}: {load().ks_status_string(s).decode()}")
+
+
+def profile_start(timing: bool = True) -> None:
+    """Reset the library's launch accounting; with timing, record event pairs."""
+    _check(load().ks_profile_start(1 if timing else 0))
+
+
+def profile_stop() -> List[dict]:
+    """Per kernel kind: launches, event time (ms), algorithmic FLOPs and bytes."""
+    arr = (KernelStat * 64)()
+    n = ctypes.c_int32()
+    _check(load().ks_profile_stop(arr, 64, ctypes.byref(n)))
+    return [{"name": arr[i].name.decode(), "launches": arr[i].launches,
+             "total_ms": arr[i].total_ms, "flops": arr[i].flops, "bytes": arr[i].bytes}
+            for i in range(min(n.value, 64))]
+
+
+def sets_to_lists(sets: torch.Tensor, n_items: int) -> List[List[int]]:
+    """Decode the [C][words] bitmask tensor into sorted item lists (host)."""
+    s = sets.cpu().numpy().view("uint64")
+    out = []
+    for row in s:
+        items = [k for k in range(n_items) if (int(row[k >> 6]) >> (k & 63)) & 1]
+        out.append(items)
+    return out

@@ -1,0 +1,64 @@
+// Internal kernel launchers of the KnapSpec library (not part of the C ABI).
+#pragma once
+
+#include "ks_common.cuh"
+
+namespace ks {
+
+// Activation (GEMM operand) storage type: fp32 for fp32 models, bf16 otherwise.
+enum ActType { ACT_F32 = 0, ACT_BF16 = 1 };
+
+inline size_t act_bytes(int act) { return act == ACT_F32 ? 4 : 2; }
+
+// y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g  for R rows of length d.
+// x fp32; g in the weight dtype; y in the activation dtype.
+ks_status launch_rmsnorm(const float* x, const void* g, int wdt, void* y, int act, int R, int d,
+                         float eps, cudaStream_t st);
+
+// C[M][N] = A[M][K] . B[N][K]^T (+ resid[M][N]) on CUDA cores, fp32 accumulation in
+// increasing k.  A in the activation dtype, B in the weight dtype; the output is fp32
+// when out_f32, else the activation dtype.
+ks_status launch_gemm_simt(const void* A, int act, const void* B, int wdt, void* C, bool out_f32,
+                           const float* resid, int M, int N, int K, cudaStream_t st);
+
+// cos/sin table [T][hd/2] for rotate-half RoPE at positions ctx + t (fp64 angles).
+ks_status launch_rope_table(float2* cs, int T, int hd, int ctx, double base, cudaStream_t st);
+
+// In-place rotate-half RoPE of q [R][H][hd] (activation dtype), row r is token r % T.
+ks_status launch_rope_inplace(void* q, int act, const float2* cs, int R, int H, int hd, int T,
+                              cudaStream_t st);
+
+// g[i] = silu(g[i]) * u[i] for n elements (activation dtype, in place).
+ks_status launch_swiglu_inplace(void* g, const void* u, int act, long long n, cudaStream_t st);
+
+// o[r][h] = softmax(q[r][h] . K[0..ctx+t]^T / sqrt(hd)) . V  with t = r % T and kv head
+// h / (Hq / Hkv).  q, o: [R][Hq][hd] activation dtype; kc, vc: one layer's cache
+// [rows][Hkv][hd] in the weight dtype.  CUDA-core version.
+ks_status launch_attention_simt(const void* q, int act, const void* kc, const void* vc, int wdt,
+                                int R, int T, int Hq, int Hkv, int hd, int ctx, void* o,
+                                cudaStream_t st);
+
+// dst[c] = src for c in [0, n_copies), each copy n_elems floats.
+ks_status launch_broadcast(float* dst, const float* src, int n_copies, long long n_elems,
+                           cudaStream_t st);
+
+// ---- DP step kernels (ks_select.cu)
+ks_status launch_select(const float* prev, const float* exec, const float* target, int C, int T,
+                        int d, int w, float* cur, float* val, uint8_t* bp, float* cos_s,
+                        float* cos_e, cudaStream_t st);
+
+struct ItemTable {
+  static constexpr int kMaxItems = 256;
+  int32_t w[kMaxItems];
+  double t[kMaxItems];
+};
+
+ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* t,
+                             const ItemTable* tab, int n_items, int C, uint64_t* sets,
+                             int32_t* used_w, double* t_draft, int32_t* status, cudaStream_t st);
+
+ks_status launch_tpt(const float* values, const double* t_draft, int C, double t_target,
+                     int gamma_max, double lo, double scale, double amax, double* tpt,
+                     int32_t* best, double* best_tpt, cudaStream_t st);
+
+}  // namespace ks

@@ -161,12 +161,14 @@ def attention_core(q: np.ndarray, k: np.ndarray, v: np.ndarray, ctx: int,
         for m0 in range(0, M, rows_per_chunk):
             m1 = min(M, m0 + rows_per_chunk)
             qg = q[m0:m1, :, g * group:(g + 1) * group, :]     # [m, T, group, hd]
-            s = np.einsum("mtgd,nd->mtgn", qg, kg) * scale
+            mm = m1 - m0
+            s = (qg.reshape(-1, hd) @ kg.T).reshape(mm, T, group, n_keys) * scale
             s = np.where(allowed[None, :, None, :], s, -np.inf)
             s = s - s.max(axis=-1, keepdims=True)
             p = np.exp(s)
             p = p / p.sum(axis=-1, keepdims=True)
-            out[m0:m1, :, g * group:(g + 1) * group, :] = np.einsum("mtgn,nd->mtgd", p, vg)
+            out[m0:m1, :, g * group:(g + 1) * group, :] = \
+                (p.reshape(-1, n_keys) @ vg).reshape(mm, T, group, hd)
     return out
 
 

@@ -1,0 +1,148 @@
+"""The C-ABI library loads, exports every declared entry point, and its host-only
+calls (weight quantisation, sizes, argument checks) behave -- no GPU needed."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+from knapsack_layer_selection_b200 import binding as B
+from knapsack_layer_selection_b200 import build as BUILD
+from knapsack_layer_selection_b200 import workloads as W
+from oracle import ks_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "knapspec.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"KS_API\s+[\w\s\*]+?\b(ks_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in B.version()
+    assert lib.ks_status_string(0) == b"ok"
+    assert lib.ks_status_string(5) == b"device wait timed out"
+
+
+def test_quantize_matches_golden(lib):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "quantized_weights.json")))
+    for c in g["cases"]:
+        t = [c["t_attn"], c["t_mlp"]] * c["layers"]
+        assert B.quantize_weights(t, c["bins"]) == [c["w_attn"], c["w_mlp"]] * c["layers"]
+
+
+def test_quantize_matches_oracle_on_random_latencies(lib):
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for _ in range(200):
+        n = int(rng.integers(1, 40))
+        t = rng.uniform(0.05, 50.0, n).tolist()
+        bins = int(rng.integers(1, 2000))
+        assert B.quantize_weights(t, bins) == O.quantize_weights(t, bins)
+    # exact halves round up
+    assert B.quantize_weights([2.5, 1.5], 4) == [3, 2]
+
+
+def test_quantize_rejects_bad_input(lib):
+    with pytest.raises(B.KnapSpecError, match="invalid argument"):
+        B.quantize_weights([1.0, 0.0], 4)
+    with pytest.raises(B.KnapSpecError):
+        B.quantize_weights([1.0], 0)
+
+
+def test_solve_cells_and_workspace_sizes(lib):
+    wl = W.WORKLOADS["llama3_8b_8k"]
+    prm = B.params(wl.gamma_max, wl.n_bins)
+    assert B.solve_cells(wl.latencies(), prm) == 513
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                     wl.ffn, wl.rms_eps, wl.rope_base, wl.wdtype)
+    ws = B.workspace_size(m, 513, wl.T)
+    R = 513 * wl.T
+    # three fp32 state buffers plus the bf16 operands dominate
+    assert ws >= 3 * R * wl.d_model * 4 + R * (wl.d_model + 2 * wl.q_dim + 2 * wl.ffn) * 2
+    assert ws < 4 * 1024 ** 3
+
+
+@pytest.mark.parametrize("name", W.WORKLOAD_ORDER)
+def test_every_workload_is_accepted(lib, name):
+    wl = W.WORKLOADS[name]
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                     wl.ffn, wl.rms_eps, wl.rope_base, wl.wdtype)
+    C = B.solve_cells(wl.latencies(), B.params(wl.gamma_max, wl.n_bins))
+    assert C == sum(O.quantize_weights(wl.latencies(), wl.n_bins)) + 1
+    assert B.workspace_size(m, C, wl.T) > 0
+
+
+def test_model_checks(lib):
+    bad = B.model_desc(2, 100, 4, 4, 64, 128, 1e-6, 1e4, "f32")   # d not a multiple of 64
+    with pytest.raises(B.KnapSpecError, match="d_model"):
+        B.workspace_size(bad, 10, 4)
+    bad = B.model_desc(2, 128, 4, 3, 64, 128, 1e-6, 1e4, "f32")   # Hq not a multiple of Hkv
+    with pytest.raises(B.KnapSpecError, match="n_kv_heads"):
+        B.workspace_size(bad, 10, 4)
+    bad = B.model_desc(2, 128, 4, 4, 96, 128, 1e-6, 1e4, "f32")   # head_dim 96
+    with pytest.raises(B.KnapSpecError, match="head_dim"):
+        B.workspace_size(bad, 10, 4)
+    good = B.model_desc(2, 128, 4, 4, 64, 128, 1e-6, 1e4, "f32")
+    with pytest.raises(B.KnapSpecError, match="T must"):
+        B.workspace_size(good, 10, 0)
+
+
+def test_solve_rejects_null_and_short_workspace_before_any_launch(lib):
+    """Argument errors come back as status codes without touching the device."""
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    prm = B.params(4, 8)
+    t = (ctypes.c_double * 2)(1.0, 1.0)
+    res = B.Result()
+    st = lib.ks_solve(ctypes.byref(m), None, None, 4, None, None, None, t, ctypes.byref(prm),
+                      None, 0, ctypes.byref(res), None)
+    assert st == 1
+    # a result without its required buffers is rejected
+    x0 = ctypes.c_void_p(256)
+    st = lib.ks_solve(ctypes.byref(m), None, None, 4, x0, None, None, t, ctypes.byref(prm),
+                      None, 0, ctypes.byref(res), None)
+    assert st == 1 and b"result needs" in lib.ks_last_error()
+    # everything present but the workspace is too small
+    layers = (B.LayerWeights * 1)()
+    for f, _ in B.LayerWeights._fields_:
+        setattr(layers[0], f, 256)
+    cache = B.CacheDesc(256, 256, 16, 8)
+    res = B.Result(*([256] * 12))
+    st = lib.ks_solve(ctypes.byref(m), layers, ctypes.byref(cache), 4, x0, None, None, t,
+                      ctypes.byref(prm), ctypes.c_void_p(256), 1024, ctypes.byref(res), None)
+    assert st == 3 and b"workspace" in lib.ks_last_error()
+    # cache too short for ctx + T
+    cache = B.CacheDesc(256, 256, 10, 8)
+    st = lib.ks_solve(ctypes.byref(m), layers, ctypes.byref(cache), 4, x0, None, None, t,
+                      ctypes.byref(prm), ctypes.c_void_p(256), 1 << 40, ctypes.byref(res), None)
+    assert st == 1 and b"cache_rows" in lib.ks_last_error()
+
+
+def test_step_calls_reject_bad_arguments(lib):
+    st = lib.ks_select_step(None, None, None, 4, 4, 64, 1, None, None, None, None, None, None)
+    assert st == 1
+    p = ctypes.c_void_p(256)
+    st = lib.ks_select_step(p, p, p, 4, 4, 64, 0, ctypes.c_void_p(512), p, p, None, None, None)
+    assert st == 1   # w must be >= 1
+    st = lib.ks_reconstruct(p, p, p, 300, 4, p, None, None, None, None)
+    assert st == 1   # more than 256 items
+    prm = B.params(0, 8)
+    st = lib.ks_tpt_argmax(p, p, 4, 10.0, ctypes.byref(prm), None, p, None, None)
+    assert st == 1   # gamma_max must be >= 1
