@@ -188,6 +188,31 @@ KS_API ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer
                                ks_stream_t stream);
 
 /*
+ * ks_reference_forward without a workspace argument (the paper has no
+ * counterpart; this is a deployment convenience).  Same inputs, outputs and
+ * arithmetic as ks_reference_forward, for callers that cannot allocate device
+ * memory at the point where they need the reference states -- for example a
+ * serving loop that refreshes X^(i) between decode steps while its memory
+ * pool forbids new device allocations, or a plugin host that hands out only
+ * input and output buffers.  The library allocates nothing here either: the
+ * scratch is one fixed 8 MiB device array inside the library, which every GPU
+ * that loads the library holds until the process exits.
+ *  - The first call on a device looks up that array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Sizes whose scratch exceeds 8 MiB (T * (d_model + 2 Hq hd + 2 ffn) *
+ *    bytes-per-element, plus alignment) are rejected with KS_ERR_UNSUPPORTED.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents; every byte a call reads it has written first, so nothing needs
+ *    clearing.  Calls that overlap on the GPU (other streams, other threads)
+ *    race on the array: serialise them.
+ */
+KS_API ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
+                                              const ks_layer_weights* layers,
+                                              const ks_cache_desc* cache, int32_t T,
+                                              const float* x0, float* ref_out,
+                                              ks_stream_t stream);
+
+/*
  * a4 -- one DP row's select step (Eq. 7/8): for every cell b in 0 .. C-1,
  *   s = meancos(prev[b], target), e = meancos(exec[b - w], target) if b >= w,
  *   cur[b] = exec[b - w] if e > s else prev[b];  val[b], bp[b] record the choice.

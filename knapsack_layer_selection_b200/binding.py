@@ -63,7 +63,7 @@ class KernelStat(ctypes.Structure):
 EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weights",
            "ks_workspace_size", "ks_sublayer_forward", "ks_reference_forward",
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
-           "ks_profile_start", "ks_profile_stop"]
+           "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc"]
 
 _lib = None
 
@@ -92,6 +92,7 @@ def load() -> ctypes.CDLL:
         "ks_solve": ([P, P, P, I32, P, P, P, P, P, P, SZ, P, P], ctypes.c_int),
         "ks_solve_cells": ([I32, P, P, P, ctypes.POINTER(I32)], ctypes.c_int),
         "ks_profile_start": ([I32], ctypes.c_int),
+        "ks_reference_forward_noalloc": ([P, P, P, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -191,6 +192,15 @@ def reference_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, x0: to
                                        _dev(x0, torch.float32, "x0"),
                                        _dev(ref_out, torch.float32, "ref_out"),
                                        _dev(ws, name="workspace"), ws.numel(), _stream()))
+
+
+def reference_forward_noalloc(model: ModelDesc, layers, cache: CacheDesc, T: int,
+                              x0: torch.Tensor, ref_out: torch.Tensor) -> None:
+    """ks_reference_forward using the library's fixed scratch array (no workspace)."""
+    _check(load().ks_reference_forward_noalloc(ctypes.byref(model), layers, ctypes.byref(cache),
+                                               T, _dev(x0, torch.float32, "x0"),
+                                               _dev(ref_out, torch.float32, "ref_out"),
+                                               _stream()))
 
 
 def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:

@@ -10,6 +10,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -220,6 +221,59 @@ static ks_status reference_chain(const Ctx& c, const float* x0, float* ref) {
     KS_CUDA_TRY(cudaMemcpyAsync(ref, x0, cell * sizeof(float), cudaMemcpyDeviceToDevice, c.st));
   for (int k = 0; k < 2 * c.m->n_layers; ++k)
     KS_TRY(sublayer(c, k, ref + k * cell, 1, ref + (k + 1) * cell));
+  return KS_OK;
+}
+
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch for ks_reference_forward_noalloc: a fixed device array that every GPU
+// loading this library holds until the process exits.  Host code must not use
+// the symbol itself as a pointer (that is a host-side stand-in); it asks the
+// runtime for the device address once per device.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+constexpr int kMaxDevices = 64;
+
+// Carves only the per-call operands of the sublayer forward (x^, q, o, gate,
+// up, RoPE table) for R = T rows; returns the bytes needed.
+static size_t carve_sublayer_only(const ks_model_desc* m, long long T, char* base, Workspace* w) {
+  const int act = m->wdtype == KS_F32 ? ACT_F32 : ACT_BF16;
+  const size_t ab = act_bytes(act);
+  const long long d = m->d_model, qd = (long long)m->n_q_heads * m->head_dim, F = m->ffn;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  };
+  *w = Workspace{};
+  w->xh = take(T * d * ab);
+  w->q = take(T * qd * ab);
+  w->att = take(T * qd * ab);
+  w->gb = take(T * F * ab);
+  w->ub = take(T * F * ab);
+  w->rope = (float2*)take(T * (m->head_dim / 2) * sizeof(float2));
+  w->total = off;
+  return off;
+}
+
+// Device address of g_static_scratch on the current device, looked up on the
+// first call for that device (with the device current) and cached.
+static ks_status static_scratch(char** out) {
+  int dev = -1;
+  KS_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(KS_ERR_UNSUPPORTED, "device index above 63");
+  static std::mutex mu;
+  static char* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(KS_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") +
+                                   cudaGetErrorString(e));
+    addr[dev] = (char*)p;
+  }
+  *out = addr[dev];
   return KS_OK;
 }
 
@@ -456,6 +510,36 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
                     params->alpha_scale, params->alpha_max, out->tpt, out->best, out->best_tpt,
                     st));
   return KS_OK;
+}
+
+ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
+                                       const ks_layer_weights* layers,
+                                       const ks_cache_desc* cache, int32_t T, const float* x0,
+                                       float* ref_out, ks_stream_t stream) {
+  KS_TRY(check_model(model));
+  KS_TRY(check_T(T));
+  KS_TRY(check_cache(model, cache, T));
+  KS_TRY(check_layers(model, layers));
+  if (!x0 || !ref_out) return fail(KS_ERR_INVALID_ARG, "x0 / ref_out is NULL");
+  Workspace w;
+  const size_t need = carve_sublayer_only(model, T, nullptr, &w);
+  if (need > kStaticScratchBytes)
+    return fail(KS_ERR_UNSUPPORTED,
+                "reference_forward_noalloc: this model and T need " + std::to_string(need) +
+                    " bytes of scratch, above the fixed " + std::to_string(kStaticScratchBytes) +
+                    "; use ks_reference_forward with a workspace");
+  char* base = nullptr;
+  KS_TRY(static_scratch(&base));
+  Ctx c;
+  c.m = model;
+  c.layers = layers;
+  c.cache = cache;
+  c.T = T;
+  c.act = model->wdtype == KS_F32 ? ACT_F32 : ACT_BF16;
+  carve_sublayer_only(model, T, base, &c.ws);
+  c.st = (cudaStream_t)stream;
+  KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
+  return reference_chain(c, x0, ref_out);
 }
 
 }  // extern "C"
