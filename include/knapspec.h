@@ -164,6 +164,24 @@ KS_API ks_status ks_quantize_weights(const double* t, int32_t n_items, int32_t n
 KS_API ks_status ks_workspace_size(const ks_model_desc* model, int32_t n_cells, int32_t T, size_t* bytes);
 
 /*
+ * Device status of the last ks_sublayer_forward / ks_reference_forward call
+ * that used this workspace: its first 4 bytes hold 0, or the ks_status a
+ * kernel reported (KS_ERR_TIMEOUT when a bounded wait gave up).  Copies them
+ * to *host_status and synchronises the stream.
+ */
+KS_API ks_status ks_workspace_status(const void* workspace, int32_t* host_status, ks_stream_t stream);
+
+/*
+ * Utility -- the tensor-core GEMM the sublayers are built on:
+ * C[M][N] = A[M][K] . B[N][K]^T (+ resid[M][N]).  A, B: device bf16
+ * row-major; C, resid: device fp32 [M][N]; resid may be NULL.  K must be a
+ * multiple of 64 and N of 256 (else KS_ERR_UNSUPPORTED).  status: device [1]
+ * word for a timed-out wait, or NULL.  Exposed for testing and reuse.
+ */
+KS_API ks_status ks_gemm_bf16(const void* A, const void* B, float* C, const float* resid,
+                              int32_t M, int32_t N, int32_t K, int32_t* status, ks_stream_t stream);
+
+/*
  * a2 / a3 -- one sublayer on a batch of E states (Eq. 7's "execute" branch).
  * Attention (item 2l): H + Wo . Attn(RoPE(Wq . RMSNorm(H))) with causal GQA
  * over the cache; MLP (item 2l+1): H + W_down (silu(W_gate x) * W_up x),
@@ -205,6 +223,8 @@ KS_API ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer
  *    contents; every byte a call reads it has written first, so nothing needs
  *    clearing.  Calls that overlap on the GPU (other streams, other threads)
  *    race on the array: serialise them.
+ *  - This path has no status word: a bounded device wait that gives up is not
+ *    reported here (use ks_reference_forward to see it).
  */
 KS_API ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
                                               const ks_layer_weights* layers,

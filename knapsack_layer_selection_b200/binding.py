@@ -63,7 +63,8 @@ class KernelStat(ctypes.Structure):
 EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weights",
            "ks_workspace_size", "ks_sublayer_forward", "ks_reference_forward",
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
-           "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc"]
+           "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
+           "ks_workspace_status", "ks_gemm_bf16"]
 
 _lib = None
 
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
         "ks_solve_cells": ([I32, P, P, P, ctypes.POINTER(I32)], ctypes.c_int),
         "ks_profile_start": ([I32], ctypes.c_int),
         "ks_reference_forward_noalloc": ([P, P, P, I32, P, P, P], ctypes.c_int),
+        "ks_workspace_status": ([P, ctypes.POINTER(I32), P], ctypes.c_int),
+        "ks_gemm_bf16": ([P, P, P, P, I32, I32, I32, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -201,6 +204,24 @@ def reference_forward_noalloc(model: ModelDesc, layers, cache: CacheDesc, T: int
                                                T, _dev(x0, torch.float32, "x0"),
                                                _dev(ref_out, torch.float32, "ref_out"),
                                                _stream()))
+
+
+def workspace_status(ws: torch.Tensor) -> int:
+    """Device status word of the last sublayer/reference call on this workspace."""
+    out = ctypes.c_int32()
+    _check(load().ks_workspace_status(_dev(ws, name="workspace"), ctypes.byref(out), _stream()))
+    return out.value
+
+
+def gemm_bf16(A: torch.Tensor, Bw: torch.Tensor, C: torch.Tensor,
+              resid: Optional[torch.Tensor] = None,
+              status: Optional[torch.Tensor] = None) -> None:
+    """C = A . Bw^T (+ resid) on the tensor cores (A [M][K], Bw [N][K] bf16; C fp32)."""
+    M, K = A.shape
+    N = Bw.shape[0]
+    _check(load().ks_gemm_bf16(_dev(A, torch.bfloat16, "A"), _dev(Bw, torch.bfloat16, "B"),
+                               _dev(C, torch.float32, "C"), _dev(resid, torch.float32, "resid"),
+                               M, N, K, _dev(status, torch.int32, "status"), _stream()))
 
 
 def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:

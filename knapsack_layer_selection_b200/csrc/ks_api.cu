@@ -101,6 +101,7 @@ static Workspace carve(const ks_model_desc* m, long long C, long long T, char* b
     off += align_up(bytes);
     return p;
   };
+  w.status = (int32_t*)take(256);   // first: the device status word of the last call
   w.prev = (float*)take(R * d * 4);
   w.cur = (float*)take(R * d * 4);
   w.exec = (float*)take(R * d * 4);
@@ -114,7 +115,6 @@ static Workspace carve(const ks_model_desc* m, long long C, long long T, char* b
   w.val = (float*)take(C * 4);
   w.t_draft = (double*)take(C * 8);
   w.rope = (float2*)take(T * (m->head_dim / 2) * sizeof(float2));
-  w.status = (int32_t*)take(256);
   w.total = off;
   return w;
 }
@@ -127,6 +127,7 @@ struct Ctx {
   int T;
   int act;
   Workspace ws;
+  int32_t* status;   // device word a timed-out wait reports into (may be NULL)
   cudaStream_t st;
 };
 
@@ -159,7 +160,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                    tc ? 1 : 2);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.xh, L.wq, nullptr, c.ws.q, nullptr, R, qd, d, EPI_ROPE_BF16, c.ws.rope,
-                       c.T, m->head_dim, c.st));
+                       c.T, m->head_dim, c.status, c.st));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.xh, c.act, L.wq, m->wdtype, c.ws.q, false, nullptr, R, qd, d,
                                 c.st));
@@ -181,7 +182,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                    (Rd * qd + (double)d * qd) * ab + Rd * d * 8.0);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.att, L.wo, nullptr, out, in, R, d, qd, EPI_RESID_F32, nullptr, c.T,
-                       m->head_dim, c.st));
+                       m->head_dim, c.status, c.st));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.att, c.act, L.wo, m->wdtype, out, true, in, R, d, qd, c.st));
       }
@@ -193,7 +194,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                    (Rd * d + 2.0 * F * d) * ab + Rd * F * ab, tc ? 1 : 3);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.xh, L.w_gate, L.w_up, c.ws.gb, nullptr, R, F, d, EPI_SWIGLU_BF16,
-                       nullptr, c.T, m->head_dim, c.st));
+                       nullptr, c.T, m->head_dim, c.status, c.st));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.xh, c.act, L.w_gate, m->wdtype, c.ws.gb, false, nullptr, R, F,
                                 d, c.st));
@@ -206,7 +207,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
       ProfScope ps(KK_GEMM_DOWN, c.st, 2.0 * Rd * d * F, (Rd * F + (double)d * F) * ab + Rd * d * 8.0);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.gb, L.w_down, nullptr, out, in, R, d, F, EPI_RESID_F32, nullptr, c.T,
-                       m->head_dim, c.st));
+                       m->head_dim, c.status, c.st));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.gb, c.act, L.w_down, m->wdtype, out, true, in, R, d, F, c.st));
       }
@@ -345,6 +346,7 @@ static ks_status make_ctx(const ks_model_desc* model, const ks_layer_weights* la
   c->T = T;
   c->act = model->wdtype == KS_F32 ? ACT_F32 : ACT_BF16;
   c->ws = carve(model, n_cells, T, (char*)workspace);
+  c->status = c->ws.status;
   c->st = st;
   return KS_OK;
 }
@@ -359,6 +361,7 @@ ks_status ks_sublayer_forward(const ks_model_desc* model, const ks_layer_weights
   if (item < 0 || item >= 2 * model->n_layers) return fail(KS_ERR_INVALID_ARG, "item out of range");
   if (E < 0) return fail(KS_ERR_INVALID_ARG, "E must be >= 0");
   if (E > 0 && (!states_in || !states_out)) return fail(KS_ERR_INVALID_ARG, "states are NULL");
+  KS_CUDA_TRY(cudaMemsetAsync(c.status, 0, sizeof(int32_t), c.st));
   KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
   return sublayer(c, item, states_in, E, states_out);
 }
@@ -370,6 +373,7 @@ ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer_weight
   Ctx c;
   KS_TRY(make_ctx(model, layers, cache, T, 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
   if (!x0 || !ref_out) return fail(KS_ERR_INVALID_ARG, "x0 / ref_out is NULL");
+  KS_CUDA_TRY(cudaMemsetAsync(c.status, 0, sizeof(int32_t), c.st));
   KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
   return reference_chain(c, x0, ref_out);
 }
@@ -460,6 +464,7 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   const int C = (int)(K + 1);
   Ctx c;
   KS_TRY(make_ctx(model, layers, cache, T, C, workspace, workspace_bytes, (cudaStream_t)stream, &c));
+  c.status = out->status;
   const cudaStream_t st = c.st;
   const long long cell = (long long)T * model->d_model;
 
@@ -537,9 +542,26 @@ ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
   c.T = T;
   c.act = model->wdtype == KS_F32 ? ACT_F32 : ACT_BF16;
   carve_sublayer_only(model, T, base, &c.ws);
+  c.status = nullptr;
   c.st = (cudaStream_t)stream;
   KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
   return reference_chain(c, x0, ref_out);
+}
+
+ks_status ks_gemm_bf16(const void* A, const void* B, float* C, const float* resid, int32_t M,
+                       int32_t N, int32_t K, int32_t* status, ks_stream_t stream) {
+  if (!A || !B || !C) return fail(KS_ERR_INVALID_ARG, "gemm: NULL pointer");
+  if (M < 0 || N < 1 || K < 1) return fail(KS_ERR_INVALID_ARG, "gemm: bad size");
+  return tc_gemm(A, B, nullptr, C, resid, M, N, K, resid ? EPI_RESID_F32 : EPI_STORE_F32, nullptr,
+                 1, 64, status, (cudaStream_t)stream);
+}
+
+ks_status ks_workspace_status(const void* workspace, int32_t* host_status, ks_stream_t stream) {
+  if (!workspace || !host_status) return fail(KS_ERR_INVALID_ARG, "workspace_status: NULL pointer");
+  KS_CUDA_TRY(cudaMemcpyAsync(host_status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                              (cudaStream_t)stream));
+  KS_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  return KS_OK;
 }
 
 }  // extern "C"

@@ -1,17 +1,387 @@
-// Tensor-core GEMM (placeholder until the tcgen05 kernel lands): the bf16 path
-// runs on the CUDA-core kernels.
+// Tensor-core GEMM of the bf16 sublayer forward on sm_100a:
+//   C[M][N] = A[M][K] . B[N][K]^T   (A = activations, B = a [out][in] weight)
+// with the sublayer's elementwise work fused into the epilogue (RoPE on the
+// query projection, SwiGLU on the gate/up projection, the fp32 residual add on
+// the output/down projections).  These are the contractions the KnapSpec DP
+// runs for every budget cell that executes an item (KnapSpec review page,
+// "What carries the argument": Attention and MLP sublayers are the items).
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialised):
+//   warp 0  -- TMA producer: 128x64 A tile and 256x64 B tile per stage, 128-byte
+//              swizzle, 4-stage ring of 48 KB stages guarded by full/empty mbarriers;
+//   warp 1  -- allocates 512 TMEM columns and one lane issues tcgen05.mma
+//              (M=128, N=256, K=16) into one of two 256-column fp32 accumulators;
+//   warps 2-5 -- epilogue: tcgen05.ld 32 columns at a time from their 32-lane
+//              quarter, apply the fused epilogue, store to global memory.
+// The accumulator double buffer lets the epilogue of tile i overlap the MMAs of
+// tile i+1.  Tiles are walked M-fastest so CTAs running together share one
+// weight tile through L2.  No split-K: every output is the same fixed-order
+// sum over K whatever M is, so a row's result does not depend on its batch.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "ks_sm100.cuh"
 #include "ks_tc.cuh"
 
 namespace ks {
 
-bool use_tensor_cores(const ks_model_desc* m) {
-  (void)m;
-  return false;
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_BYTES = BN * BK * 2;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;               // two 256-column fp32 accumulators
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+struct SharedTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
-ks_status tc_gemm(const void*, const void*, const void*, void*, const float*, int, int, int, int,
-                  const float2*, int, int, cudaStream_t) {
-  return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM not built");
+// Stores 32 consecutive bf16 values (64 bytes) at p (16-byte aligned).
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float (&v)[32]) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    q[j] = make_uint4(pack_bf16(v[8 * j + 0], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                      pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
+}
+
+struct GemmParams {
+  void* out;
+  const float* resid;
+  const float2* rope_cs;
+  int32_t* status;
+  int M, N_out, K;
+  int tiles_m, tiles_n;
+  int T, head_dim;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, const GemmParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  SharedTail* tail = reinterpret_cast<SharedTail*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  const int KB = p.K / BK;
+  volatile int* abort = &tail->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&tail->full[s]), 1);
+      mbar_init(smem_u32(&tail->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tail->tfull[a]), 1);
+      mbar_init(smem_u32(&tail->tempty[a]), 128);
+    }
+    mbar_init(smem_u32(&tail->drain), 1);
+    tail->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (EPI == EPI_SWIGLU_BF16) prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tail->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int m0 = (t % p.tiles_m) * BM;
+        const int tn = t / p.tiles_m;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t r = (uint32_t)(it / STAGES);
+          if (!mbar_wait(smem_u32(&tail->empty[s]), (r & 1u) ^ 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = smem_u32(&tail->full[s]);
+          const uint32_t a_dst = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_dst = a_dst + A_BYTES;
+          mbar_arrive_expect_tx(full, STAGE_BYTES);
+          tma_load_2d(a_dst, &tmA, kb * BK, m0, full);
+          if (EPI == EPI_SWIGLU_BF16) {
+            tma_load_2d(b_dst, &tmB, kb * BK, tn * (BN / 2), full);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB2, kb * BK, tn * (BN / 2), full);
+          } else {
+            tma_load_2d(b_dst, &tmB, kb * BK, tn * BN, full);
+          }
+        }
+      }
+      // never leave while a copy this thread issued may still be landing
+      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+        mbar_wait_drain(smem_u32(&tail->full[j % STAGES]), (uint32_t)(j / STAGES) & 1u, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t ar = (uint32_t)(i >> 1);
+        if (!mbar_wait(smem_u32(&tail->tempty[acc]), (ar & 1u) ^ 1u, abort, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t r = (uint32_t)(it / STAGES);
+          if (!mbar_wait(smem_u32(&tail->full[s]), r & 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t a_desc = desc_kmajor_sw128(a_addr);
+          const uint64_t b_desc = desc_kmajor_sw128(a_addr + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)   // advance 16 elements = 32 bytes = 2 units
+            mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, IDESC, (kb | k) != 0);
+          mma_commit(smem_u32(&tail->empty[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tail->tfull[acc]));
+      }
+      // wait until every MMA issued above has retired before TMEM is released
+      mma_commit(smem_u32(&tail->drain));
+      mbar_wait_drain(smem_u32(&tail->drain), 0, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    const int q = warp & 3;                       // TMEM lane quarter this warp may read
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t ar = (uint32_t)(i >> 1);
+      // the whole warp leaves together: tcgen05.ld below is warp-collective
+      const bool got = mbar_wait(smem_u32(&tail->tfull[acc]), ar & 1u, abort, p.status);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int m0 = (t % p.tiles_m) * BM;
+      const int tn = t / p.tiles_m;
+      const int row = m0 + q * 32 + lane;
+      const bool live = row < p.M;
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      float v[32], u[32];
+      if (EPI == EPI_RESID_F32 || EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
+        const int n0 = tn * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          if (!live) continue;
+          const long long off = (long long)row * p.N_out + n0 + c * 32;
+          if (EPI == EPI_STORE_BF16) {
+            store_bf16x32((__nv_bfloat16*)p.out + off, v);
+          } else {
+            float4* o = reinterpret_cast<float4*>((float*)p.out + off);
+            if (EPI == EPI_RESID_F32) {
+              const float4* rr = reinterpret_cast<const float4*>(p.resid + off);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 x = rr[j];
+                o[j] = make_float4(v[4 * j] + x.x, v[4 * j + 1] + x.y, v[4 * j + 2] + x.z,
+                                   v[4 * j + 3] + x.w);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+          }
+        }
+      } else if (EPI == EPI_SWIGLU_BF16) {
+        // columns 0..127: gate, 128..255: up, for output columns tn*128 ..
+        const int n0 = tn * (BN / 2);
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+          tmem_ld32(tbase + c * 32, v);
+          tmem_ld32(tbase + BN / 2 + c * 32, u);
+          tmem_wait_ld();
+          if (!live) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = v[j] / (1.0f + __expf(-v[j])) * u[j];
+          store_bf16x32((__nv_bfloat16*)p.out + (long long)row * p.N_out + n0 + c * 32, v);
+        }
+      } else if (EPI == EPI_ROPE_BF16) {
+        // rotate-half RoPE inside each head of this tile: column j pairs with j + hd/2
+        const int half = p.head_dim / 2;
+        const int tok = row % p.T;
+        const float2* cs = p.rope_cs + (long long)tok * half;
+        const int n0 = tn * BN;
+#pragma unroll 1
+        for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
+#pragma unroll 1
+          for (int c = 0; c < half; c += 32) {
+            tmem_ld32(tbase + h0 + c, v);
+            tmem_ld32(tbase + h0 + half + c, u);
+            tmem_wait_ld();
+            if (!live) continue;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 r = cs[c + j];
+              const float x1 = v[j], x2 = u[j];
+              v[j] = x1 * r.x - x2 * r.y;
+              u[j] = x2 * r.x + x1 * r.y;
+            }
+            __nv_bfloat16* o = (__nv_bfloat16*)p.out + (long long)row * p.N_out + n0 + h0 + c;
+            store_bf16x32(o, v);
+            store_bf16x32(o + half, u);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tail->tempty[acc]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+  });
+  return fn;
+}
+
+// Tensor map of a row-major bf16 matrix [rows][cols] read in boxes of
+// box_rows x 64 columns with the 128-byte swizzle; out-of-range rows read as 0.
+ks_status make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols,
+                    int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((uintptr_t)base % 16) return fail(KS_ERR_INVALID_ARG, "tensor base not 16-byte aligned");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return KS_OK;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int EPI>
+ks_status launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                 const GemmParams& gp, cudaStream_t st) {
+  static bool attr_set = false;
+  auto k = tc_gemm_kernel<EPI>;
+  if (!attr_set) {
+    KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    attr_set = true;
+  }
+  const int n_tiles = gp.tiles_m * gp.tiles_n;
+  const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
+  k<<<grid, THREADS, SMEM_BYTES, st>>>(a, b, b2, gp);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+}  // namespace
+
+bool use_tensor_cores(const ks_model_desc* m) { return m->wdtype == KS_BF16; }
+
+ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
+                  int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
+                  int32_t* status, cudaStream_t st) {
+  if (M <= 0) return KS_OK;
+  if (K % BK) return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: K must be a multiple of 64");
+  const int bn_out = epi == EPI_SWIGLU_BF16 ? BN / 2 : BN;
+  if (N % bn_out)
+    return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: N must be a multiple of " + std::to_string(bn_out));
+  if (epi == EPI_ROPE_BF16 && (head_dim % 64 || BN % head_dim || !rope_cs || T < 1))
+    return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: RoPE epilogue needs head_dim 64 or 128");
+  if (epi == EPI_RESID_F32 && !resid) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: resid is NULL");
+  if (epi == EPI_SWIGLU_BF16 && !B2) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: up weight is NULL");
+  CUtensorMap ta, tb, tb2;
+  KS_TRY(make_tmap(&ta, A, M, K, BM));
+  if (epi == EPI_SWIGLU_BF16) {
+    KS_TRY(make_tmap(&tb, B, N, K, BN / 2));
+    KS_TRY(make_tmap(&tb2, B2, N, K, BN / 2));
+  } else {
+    KS_TRY(make_tmap(&tb, B, N, K, BN));
+    tb2 = tb;
+  }
+  GemmParams gp;
+  gp.out = out;
+  gp.resid = resid;
+  gp.rope_cs = rope_cs;
+  gp.status = status;
+  gp.M = M;
+  gp.N_out = N;
+  gp.K = K;
+  gp.tiles_m = (M + BM - 1) / BM;
+  gp.tiles_n = N / bn_out;
+  gp.T = T;
+  gp.head_dim = head_dim;
+  switch (epi) {
+    case EPI_RESID_F32: return launch<EPI_RESID_F32>(ta, tb, tb2, gp, st);
+    case EPI_ROPE_BF16: return launch<EPI_ROPE_BF16>(ta, tb, tb2, gp, st);
+    case EPI_SWIGLU_BF16: return launch<EPI_SWIGLU_BF16>(ta, tb, tb2, gp, st);
+    case EPI_STORE_BF16: return launch<EPI_STORE_BF16>(ta, tb, tb2, gp, st);
+    case EPI_STORE_F32: return launch<EPI_STORE_F32>(ta, tb, tb2, gp, st);
+  }
+  return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: unknown epilogue");
 }
 
 }  // namespace ks
