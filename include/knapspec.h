@@ -182,6 +182,19 @@ KS_API ks_status ks_gemm_bf16(const void* A, const void* B, float* C, const floa
                               int32_t M, int32_t N, int32_t K, int32_t* status, ks_stream_t stream);
 
 /*
+ * Utility -- the tensor-core attention the Attention sublayer is built on:
+ * out[r][h] = softmax(q[r][h] . K[0 .. ctx+t]^T / sqrt(hd)) . V[0 .. ctx+t]
+ * with t = r % T and kv head h / (Hq / Hkv).  q, out: device bf16
+ * [R][Hq][head_dim]; k_layer, v_layer: device bf16 [cache_rows][Hkv][head_dim]
+ * (one layer of the cache); head_dim 64 or 128; cache_rows >= ctx + T.
+ * status: device [1] word for a timed-out wait, or NULL.
+ */
+KS_API ks_status ks_attention_bf16(const void* q, const void* k_layer, const void* v_layer,
+                                   int64_t cache_rows, int32_t R, int32_t T, int32_t Hq,
+                                   int32_t Hkv, int32_t head_dim, int32_t ctx, void* out,
+                                   int32_t* status, ks_stream_t stream);
+
+/*
  * a2 / a3 -- one sublayer on a batch of E states (Eq. 7's "execute" branch).
  * Attention (item 2l): H + Wo . Attn(RoPE(Wq . RMSNorm(H))) with causal GQA
  * over the cache; MLP (item 2l+1): H + W_down (silu(W_gate x) * W_up x),

@@ -64,7 +64,7 @@ EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weigh
            "ks_workspace_size", "ks_sublayer_forward", "ks_reference_forward",
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
            "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
-           "ks_workspace_status", "ks_gemm_bf16"]
+           "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16"]
 
 _lib = None
 
@@ -96,6 +96,7 @@ def load() -> ctypes.CDLL:
         "ks_reference_forward_noalloc": ([P, P, P, I32, P, P, P], ctypes.c_int),
         "ks_workspace_status": ([P, ctypes.POINTER(I32), P], ctypes.c_int),
         "ks_gemm_bf16": ([P, P, P, P, I32, I32, I32, P, P], ctypes.c_int),
+        "ks_attention_bf16": ([P, P, P, I64, I32, I32, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -222,6 +223,17 @@ def gemm_bf16(A: torch.Tensor, Bw: torch.Tensor, C: torch.Tensor,
     _check(load().ks_gemm_bf16(_dev(A, torch.bfloat16, "A"), _dev(Bw, torch.bfloat16, "B"),
                                _dev(C, torch.float32, "C"), _dev(resid, torch.float32, "resid"),
                                M, N, K, _dev(status, torch.int32, "status"), _stream()))
+
+
+def attention_bf16(q: torch.Tensor, k_layer: torch.Tensor, v_layer: torch.Tensor, T: int,
+                   ctx: int, out: torch.Tensor, status: Optional[torch.Tensor] = None) -> None:
+    """Tensor-core causal GQA attention: q/out [R][Hq][hd], k/v [rows][Hkv][hd] (bf16)."""
+    R, Hq, hd = q.shape
+    rows, Hkv, _ = k_layer.shape
+    _check(load().ks_attention_bf16(_dev(q, torch.bfloat16, "q"), _dev(k_layer, torch.bfloat16, "k"),
+                                    _dev(v_layer, torch.bfloat16, "v"), rows, R, T, Hq, Hkv, hd,
+                                    ctx, _dev(out, torch.bfloat16, "out"),
+                                    _dev(status, torch.int32, "status"), _stream()))
 
 
 def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:

@@ -174,8 +174,13 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
       const double kv_bytes = 2.0 * (ctx + T) * m->n_kv_heads * m->head_dim * wb;
       ProfScope ps(KK_ATTN, c.st, 4.0 * m->n_q_heads * m->head_dim * keys,
                    2.0 * Rd * qd * ab + kv_bytes);
-      KS_TRY(launch_attention_simt(c.ws.q, c.act, kc, vc, m->wdtype, R, c.T, m->n_q_heads,
-                                   m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.st));
+      if (tc) {
+        KS_TRY(tc_attention(c.ws.q, kc, vc, c.cache->cache_rows, R, c.T, m->n_q_heads,
+                            m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.status, c.st));
+      } else {
+        KS_TRY(launch_attention_simt(c.ws.q, c.act, kc, vc, m->wdtype, R, c.T, m->n_q_heads,
+                                     m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.st));
+      }
     }
     {
       ProfScope ps(KK_GEMM_O, c.st, 2.0 * Rd * d * qd,
@@ -562,6 +567,16 @@ ks_status ks_workspace_status(const void* workspace, int32_t* host_status, ks_st
                               (cudaStream_t)stream));
   KS_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
   return KS_OK;
+}
+
+ks_status ks_attention_bf16(const void* q, const void* k_layer, const void* v_layer,
+                            int64_t cache_rows, int32_t R, int32_t T, int32_t Hq, int32_t Hkv,
+                            int32_t head_dim, int32_t ctx, void* out, int32_t* status,
+                            ks_stream_t stream) {
+  if (!q || !k_layer || !v_layer || !out) return fail(KS_ERR_INVALID_ARG, "attention: NULL pointer");
+  if (R < 0 || T < 1 || Hq < 1 || Hkv < 1 || ctx < 0) return fail(KS_ERR_INVALID_ARG, "attention: bad size");
+  return tc_attention(q, k_layer, v_layer, cache_rows, R, T, Hq, Hkv, head_dim, ctx, out, status,
+                      (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -1,6 +1,8 @@
 // Tensor-core (tcgen05 / TMEM / TMA) kernels of the bf16 sublayer forward.
 #pragma once
 
+#include <cuda.h>
+
 #include "ks_common.cuh"
 
 namespace ks {
@@ -23,5 +25,20 @@ bool use_tensor_cores(const ks_model_desc* m);
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
                   int32_t* status, cudaStream_t st);
+
+// Tensor map of a row-major bf16 matrix [rows][cols] (row_stride elements apart)
+// read in boxes of box_rows x box_cols with the 128-byte swizzle; reads outside
+// [rows) x [cols) return zeros.
+ks_status make_tmap_2d(CUtensorMap* m, const void* base, long long rows, long long cols,
+                       long long row_stride, int box_cols, int box_rows);
+
+// Causal GQA attention on the tensor cores: q, out [R][Hq][hd] bf16 (row r is
+// evaluation token r % T), kc/vc one layer of the cache [cache_rows][Hkv][hd]
+// bf16; token t attends to positions 0 .. ctx + t.  hd = 64 or 128.
+ks_status tc_attention(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
+                       int T, int Hq, int Hkv, int hd, int ctx, void* out, int32_t* status,
+                       cudaStream_t st);
+
+int sm_count();
 
 }  // namespace ks

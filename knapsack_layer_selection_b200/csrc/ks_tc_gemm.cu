@@ -278,6 +278,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------- host side
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -290,35 +301,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
   });
   return fn;
-}
-
-// Tensor map of a row-major bf16 matrix [rows][cols] read in boxes of
-// box_rows x 64 columns with the 128-byte swizzle; out-of-range rows read as 0.
-ks_status make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols,
-                    int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  if ((uintptr_t)base % 16) return fail(KS_ERR_INVALID_ARG, "tensor base not 16-byte aligned");
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
-  return KS_OK;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
 }
 
 template <int EPI>
@@ -339,6 +321,24 @@ ks_status launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
 
 }  // namespace
 
+ks_status make_tmap_2d(CUtensorMap* m, const void* base, long long rows, long long cols,
+                       long long row_stride, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((uintptr_t)base % 16) return fail(KS_ERR_INVALID_ARG, "tensor base not 16-byte aligned");
+  if ((row_stride * 2) % 16) return fail(KS_ERR_UNSUPPORTED, "tensor row stride not a multiple of 16 bytes");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(KS_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return KS_OK;
+}
+
 bool use_tensor_cores(const ks_model_desc* m) { return m->wdtype == KS_BF16; }
 
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
@@ -354,12 +354,12 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
   if (epi == EPI_RESID_F32 && !resid) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: resid is NULL");
   if (epi == EPI_SWIGLU_BF16 && !B2) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: up weight is NULL");
   CUtensorMap ta, tb, tb2;
-  KS_TRY(make_tmap(&ta, A, M, K, BM));
+  KS_TRY(make_tmap_2d(&ta, A, M, K, K, BK, BM));
   if (epi == EPI_SWIGLU_BF16) {
-    KS_TRY(make_tmap(&tb, B, N, K, BN / 2));
-    KS_TRY(make_tmap(&tb2, B2, N, K, BN / 2));
+    KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN / 2));
+    KS_TRY(make_tmap_2d(&tb2, B2, N, K, K, BK, BN / 2));
   } else {
-    KS_TRY(make_tmap(&tb, B, N, K, BN));
+    KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN));
     tb2 = tb;
   }
   GemmParams gp;
