@@ -1,0 +1,55 @@
+"""A small, self-contained case for profiler captures of the hot kernels.
+
+Runs one sublayer forward of a workload's shape -- the Attention item or the
+MLP item of one layer, over every budget cell that executes it in the DP
+(E = C - w_item cells x T tokens) -- a few times, with one layer of seeded
+weights and cache.  It holds about 2 GB on the device for the 8B shape, so a
+profiler can replay its kernels quickly.
+
+    python -m knapsack_layer_selection_b200.profile_case --workload llama3_8b_8k --item attn
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+
+import torch
+
+from knapsack_layer_selection_b200 import binding as B
+from knapsack_layer_selection_b200 import build as BUILD
+from knapsack_layer_selection_b200 import workloads as W
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="llama3_8b_8k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--item", choices=["attn", "mlp"], default="attn")
+    ap.add_argument("--repeat", type=int, default=2)
+    a = ap.parse_args()
+    BUILD.build()
+    full = W.WORKLOADS[a.workload]
+    wl = dataclasses.replace(full, n_layers=1)
+    inp = W.make_inputs(wl, device="cuda")
+    t = full.latencies()
+    w = B.quantize_weights(t, full.n_bins)
+    C = sum(w) + 1
+    item = 0 if a.item == "attn" else 1
+    E = C - w[item]
+    m = B.model_desc(1, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    layers = B.layer_array(inp.layers, W.torch_dtype(wl))
+    cache = B.cache_desc(inp.k_cache, inp.v_cache, wl.ctx)
+    states = W.random_states((E, wl.T, wl.d_model), 1, device="cuda")
+    out = torch.empty_like(states)
+    ws = B.workspace(m, E, wl.T)
+    for _ in range(a.repeat):
+        B.sublayer_forward(m, layers, cache, wl.T, item, states, out, ws)
+    torch.cuda.synchronize()
+    st = B.workspace_status(ws)
+    if st != 0:
+        raise SystemExit(f"device status {st}")
+    print(f"{a.workload} {a.item}: {E} cells x {wl.T} tokens, {a.repeat} forward(s) ok")
+
+
+if __name__ == "__main__":
+    main()

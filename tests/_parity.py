@@ -56,9 +56,11 @@ def taint_mask(w, bp_o, bp_g, cos_s_o, cos_e_o):
     return near, taint
 
 
-def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=None) -> Report:
+def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=None,
+                  check_argmax=True) -> Report:
     """orc: oracle Solve; gpu: dict of numpy arrays bp [n][C], values [C], sets (lists),
-    best (b, gamma), tpt grid [C][G] (optional); rows_val_gpu: [n][C] chosen values."""
+    best (b, gamma), tpt grid [C][G] (optional); rows_val_gpu: [n][C] chosen values.
+    With check_argmax=False (a budget prefix) the TPT choice is not compared."""
     bp_o = orc.dp.bp
     C = bp_o.shape[1]
     bp_g = gpu["bp"]
@@ -80,6 +82,8 @@ def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=Non
         r.val_fail += int(np.sum(e2[m] > val_tol))
     sets_g = gpu["sets"]
     r.set_mismatch_untainted = int(sum(1 for b in range(C) if ok[b] and sets_g[b] != orc.sets[b]))
+    if not check_argmax:
+        return r
     # best (S, gamma)
     bo, go = orc.best_b, orc.best_gamma
     bg, gg = int(gpu["best"][0]), int(gpu["best"][1])

@@ -1,0 +1,133 @@
+"""Full-size GPU solves of the Llama-3-8B (8k and 32k context) and Qwen3-32B
+shapes, in the launch configuration the benchmark times, checked against the
+oracle where it can compute outputs one by one:
+
+* the reference states X^(0..2L) (one chain of T tokens through every item);
+* the lowest budgets: cells 0 .. P-1 of every DP row depend only on cells
+  below P, so the oracle's DP over that prefix must agree with the GPU's
+  prefix under the near-tie/taint rule;
+
+and through properties that hold at any size: the all-execute cell reproduces
+the reference chain (value 1), reconstructed sets respect their budgets, the
+TPT choice is the grid's maximum, and a second solve is bit-identical.  The
+32k workload is also re-solved at 4k and 16k context, reporting how many
+Attention and MLP items the chosen sets skip as the context grows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from knapsack_layer_selection_b200 import binding as B
+from knapsack_layer_selection_b200 import build as BUILD
+from knapsack_layer_selection_b200 import workloads as W
+from oracle import ks_oracle as O
+from tests._parity import compare_solve
+from tests._util import oracle_model, x0_np
+
+pytestmark = pytest.mark.gpu
+
+PREFIX = {"llama3_8b_8k": 40, "llama3_8b_32k": 40, "qwen3_32b_16k": 24}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    BUILD.build()
+    return B.load()
+
+
+def run(name, ctx=None):
+    wl = W.WORKLOADS[name]
+    if ctx is not None:
+        wl = wl.with_ctx(ctx)
+    inp = W.make_inputs(W.WORKLOADS[name])          # the cache holds the largest context
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    t = wl.latencies()
+    solver = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, t,
+                      B.params(wl.gamma_max, wl.n_bins), keep_cos=True)
+    solver.solve(inp.x0)
+    torch.cuda.synchronize()
+    solver.check_status()
+    return wl, inp, solver
+
+
+def gpu_arrays(solver):
+    o = solver.out
+    bp = o.bp.cpu().numpy()
+    return {"bp": bp, "values": o.values.cpu().numpy(),
+            "sets": B.sets_to_lists(o.sets, solver.n_items), "used_w": o.used_w.cpu().numpy(),
+            "t_draft": o.t_draft.cpu().numpy(), "best": o.best.cpu().numpy(),
+            "rows": np.where(bp == 1, o.cos_exec.cpu().numpy(), o.cos_skip.cpu().numpy()),
+            "tpt": o.tpt.cpu().numpy(), "ref": o.ref_states.cpu().numpy()}
+
+
+def check_invariants(wl, solver, g):
+    C = solver.C
+    w, t = solver.w, solver.t
+    assert abs(g["values"][-1] - 1.0) <= 1e-6
+    assert g["sets"][-1] == list(range(wl.n_items))
+    for b in range(C):
+        assert g["used_w"][b] <= b
+        assert g["used_w"][b] == sum(w[k] for k in g["sets"][b])
+        acc = 0.0
+        for k in g["sets"][b]:
+            acc += t[k]
+        assert g["t_draft"][b] == acc
+    b, gm = g["best"]
+    assert g["tpt"][b, gm - 1] == np.nanmax(g["tpt"])
+    assert np.all(np.isfinite(g["values"])) and np.all(g["values"] <= 1.0 + 1e-6)
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_8k", "llama3_8b_32k", "qwen3_32b_16k"])
+def test_full_size_solve(name):
+    wl, inp, solver = run(name)
+    g = gpu_arrays(solver)
+    check_invariants(wl, solver, g)
+    # determinism
+    solver.solve(inp.x0)
+    torch.cuda.synchronize()
+    assert np.array_equal(solver.out.bp.cpu().numpy(), g["bp"])
+    assert np.array_equal(solver.out.values.cpu().numpy(), g["values"])
+
+    om = oracle_model(inp)
+    x0 = x0_np(inp)
+    ref = O.reference_states(om, x0, wl.ctx)
+    for k in range(wl.n_items + 1):
+        rel = np.linalg.norm(g["ref"][k] - ref[k]) / np.linalg.norm(ref[k])
+        assert rel < 2e-2, (k, rel)
+        assert O.meancos(g["ref"][k][None], ref[k])[0] > 1 - 1e-4
+    P = PREFIX[name]
+    orc = O.dp_solve(om, x0, wl.ctx, solver.w, solver.t, wl.gamma_max, n_cells=P, ref=ref)
+    gp = {"bp": g["bp"][:, :P], "values": g["values"][:P], "sets": g["sets"][:P],
+          "best": g["best"]}
+    rep = compare_solve(orc, gp, solver.w, 2e-3, wl.n_items, rows_val_gpu=g["rows"][:, :P],
+                        check_argmax=False)
+    print(f"\n{name}: prefix {P} of {solver.C} cells: {rep}")
+    rep.assert_ok()
+
+
+def test_long_context_resolve_shifts_the_layer_set():
+    """Re-solve the 8B shape at 4k, 16k and 32k context (the 64-step re-solve of
+    the paper's serving loop, done here at three contexts): report how the
+    chosen sets divide between skipped Attention and MLP items."""
+    report = []
+    for ctx in W.WORKLOADS["llama3_8b_32k"].contexts:
+        wl, inp, solver = run("llama3_8b_32k", ctx=ctx)
+        g = gpu_arrays(solver)
+        check_invariants(wl, solver, g)
+        b, gm = g["best"]
+        chosen = set(g["sets"][b])
+        skip_attn = sum(1 for k in range(0, wl.n_items, 2) if k not in chosen)
+        skip_mlp = sum(1 for k in range(1, wl.n_items, 2) if k not in chosen)
+        mid = solver.C // 2
+        mid_set = set(g["sets"][mid])
+        report.append((ctx, solver.w[:2], (b, gm), skip_attn, skip_mlp,
+                       sum(1 for k in range(0, wl.n_items, 2) if k not in mid_set),
+                       sum(1 for k in range(1, wl.n_items, 2) if k not in mid_set)))
+        del inp, solver
+        torch.cuda.empty_cache()
+    for r in report:
+        print(f"\nctx {r[0]}: w(Attn, MLP) = {r[1]}, best (b, gamma) = {r[2]}, best set skips "
+              f"{r[3]} Attn / {r[4]} MLP; budget K/2 skips {r[5]} Attn / {r[6]} MLP")
