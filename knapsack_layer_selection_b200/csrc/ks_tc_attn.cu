@@ -13,14 +13,20 @@
 //   warp 0    -- TMA: the Q tile once, then K and V blocks of 128 keys into a
 //                2-stage ring (64-column panels, 128-byte swizzle);
 //   warp 1    -- TMEM owner; one lane issues S_j = Q K_j^T (M=128, N=128) into
-//                one of two S buffers, and O_j = P_j V_j (M=128, N=hd, V read
-//                MN-major straight from the cache layout) into one of two O
-//                buffers, in the order S_0, S_1, O_0, S_2, O_1, ... so the
+//                one of two S buffers and O += P_j V_j (M=128, N=hd, V read
+//                MN-major straight from the cache layout) into one TMEM
+//                accumulator, in the order S_0, S_1, PV_0, S_2, PV_1, ... so the
 //                softmax of block j+1 overlaps the P.V product of block j;
-//   warps 2-5 -- one thread per query row: online softmax (running max and sum
-//                in the exp2 domain), P_j to shared memory as bf16 in the
-//                swizzled K-major layout the MMA reads, and O accumulated in
-//                registers as O <- O * alpha + O_j.
+//   warps 2-5 -- one thread per query row: the scores of a block go from TMEM to
+//                registers once; the running maximum is kept "stale": P is taken
+//                relative to a reference maximum that moves only when the row's
+//                maximum grows by more than 2^8, and only then is the row's O in
+//                TMEM rescaled (after the previous P.V has landed).  exp2 runs
+//                on the MUFU unit for three of every four scores and as a cubic
+//                on the FMA pipe for the fourth.  Only blocks that reach past
+//                position ctx are masked.  P goes to shared memory as bf16 in the
+//                swizzled K-major layout the MMA reads; O is normalised by the
+//                running sum once, at the end.
 // Every row uses the same block order and the same arithmetic whatever the
 // batch, so a row's output does not depend on the other rows.
 #include <cuda.h>
@@ -50,7 +56,7 @@ struct Cfg {
   static constexpr int OFF_TAIL = OFF_P + 2 * P_BYTES;
   static constexpr int SMEM = OFF_TAIL + 256 + 1024;
   static constexpr int TMEM_S = 0;                    // S buffers: columns [0, 2*BN)
-  static constexpr int TMEM_O = 2 * BN;               // O buffers: [2*BN, 2*BN + 2*HD)
+  static constexpr int TMEM_O = 2 * BN;               // O accumulator: [2*BN, 2*BN + HD)
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, HD) | (1u << 16);   // B (V) MN-major
@@ -59,7 +65,7 @@ struct Cfg {
 struct Tail {
   uint64_t q_full;
   uint64_t k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full[2], s_free[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -76,6 +82,35 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x as 2^floor(x) * p(x - floor(x)); p is a cubic fitted to 2^f on [0, 1)
+// for minimal relative error (7.5e-5, far below the bf16 rounding of P).
+// Runs on the FMA pipe; used for a share of the scores to unload MUFU.
+__device__ __forceinline__ float exp2_cubic(float x) {
+  x = fmaxf(x, -125.0f);   // keeps the exponent field of the result positive
+  const float fl = floorf(x);
+  const float f = x - fl;
+  const float p = fmaf(fmaf(fmaf(0.07802403f, f, 0.22606707f), f, 0.69583398f), f, 0.99992514f);
+  return __int_as_float(__float_as_int(p) + ((int)fl << 23));
+}
+
+// 32 consecutive fp32 columns into this thread's TMEM lane (32x32b shape, x32).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
+      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
+      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
+      "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -128,8 +163,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&tail->s_full[s]), 1);
       mbar_init(smem_u32(&tail->s_free[s]), 128);
       mbar_init(smem_u32(&tail->p_full[s]), 128);
-      mbar_init(smem_u32(&tail->o_full[s]), 1);
-      mbar_init(smem_u32(&tail->o_free[s]), 128);
+      mbar_init(smem_u32(&tail->o_done[s]), 1);
     }
     mbar_init(smem_u32(&tail->drain), 1);
     tail->abort = 0;
@@ -205,8 +239,7 @@ __global__ void __launch_bounds__(192, 1)
           const int s = i & 1;
           const uint32_t r = (uint32_t)(i >> 1);
           if (!mbar_wait(smem_u32(&tail->p_full[s]), r & 1u, abort, p.status) ||
-              !mbar_wait(smem_u32(&tail->v_full[s]), r & 1u, abort, p.status) ||
-              !mbar_wait(smem_u32(&tail->o_free[s]), (r & 1u) ^ 1u, abort, p.status)) {
+              !mbar_wait(smem_u32(&tail->v_full[s]), r & 1u, abort, p.status)) {
             ok = false;
             break;
           }
@@ -218,9 +251,9 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t a = desc_kmajor_sw128(pb + (kk / 4) * C::P_PANEL) + 2 * (kk % 4);
             // 16 keys = 16 rows of 128 bytes further along K
             const uint64_t b = desc_mnmajor_sw128(vst + kk * 16 * 128, C::KV_PANEL);
-            mma_bf16(tmem + C::TMEM_O + s * HD, a, b, C::IDESC_O, kk > 0);
+            mma_bf16(tmem + C::TMEM_O, a, b, C::IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(smem_u32(&tail->o_full[s]));
+          mma_commit(smem_u32(&tail->o_done[s]));
           mma_commit(smem_u32(&tail->kv_empty[s]));
         }
       }
@@ -236,30 +269,10 @@ __global__ void __launch_bounds__(192, 1)
     const int limit = p.ctx + (live ? row % p.T : 0);   // last visible cache position
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = p.scale_log2;
-    float o[HD];
-#pragma unroll
-    for (int i = 0; i < HD; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    constexpr float kStale = 8.0f;                // rescale once the max grows by > 2^8
+    float m_ref = -INFINITY;                      // reference maximum (raw score units)
+    float l = 0.f;                                // running sum relative to m_ref
     bool ok = true;
-
-    auto correct = [&](int i, float a) -> bool {
-      const int s = i & 1;
-      if (!warp_wait(smem_u32(&tail->o_full[s]), (uint32_t)(i >> 1) & 1u, abort, p.status))
-        return false;
-      tc_fence_after();
-      float v[32];
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        tmem_ld32(tmem + lane_off + C::TMEM_O + s * HD + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[c * 32 + e] = fmaf(o[c * 32 + e], a, v[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&tail->o_free[s]));
-      return true;
-    };
-
     for (int j = 0; j < J; ++j) {
       const int s = j & 1;
       if (!warp_wait(smem_u32(&tail->s_full[s]), (uint32_t)(j >> 1) & 1u, abort, p.status)) {
@@ -269,37 +282,72 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t ts = tmem + lane_off + C::TMEM_S + s * C::BN;
       const int key0 = j * C::BN;
-      float v[32];
-      // pass 1: block maximum of the scaled scores over visible keys
-      float bmax = -INFINITY;
+      const bool masked = key0 + C::BN - 1 > p.ctx;   // some key may be past a row's window
+      float sc[C::BN];
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        tmem_ld32(ts + c * 32, v);
-        tmem_wait_ld();
+      for (int c = 0; c < C::BN / 32; ++c)
+        tmem_ld32(ts + c * 32, *reinterpret_cast<float(*)[32]>(&sc[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tail->s_free[s]));    // S buffer may be overwritten now
+      if (masked) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = (key0 + c * 32 + e <= limit) ? v[e] * sl2 : -INFINITY;
-          bmax = fmaxf(bmax, x);
+        for (int e = 0; e < C::BN; ++e)
+          if (key0 + e > limit) sc[e] = -INFINITY;
+      }
+      float bmax = sc[0];
+#pragma unroll
+      for (int e = 1; e < C::BN; ++e) bmax = fmaxf(bmax, sc[e]);
+      const bool grow = (bmax - m_ref) * sl2 > kStale;   // true on the first block
+      if (__any_sync(0xffffffffu, grow && j > 0)) {
+        // rescale this warp's O rows once the previous P.V has landed in TMEM
+        const int i = j - 1;
+        if (!warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort,
+                       p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float a = grow ? ex2((m_ref - bmax) * sl2) : 1.0f;
+        float v[32];
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          const uint32_t to = tmem + lane_off + C::TMEM_O + c * 32;
+          tmem_ld32(to, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= a;
+          tmem_st32(to, v);
+        }
+        tmem_wait_st();
+        l *= a;
+      }
+      if (grow) m_ref = bmax;
+      // P_j into shared buffer s: the P.V that last read it (block j-2) must be done
+      if (j >= 2) {
+        const int i = j - 2;
+        if (!warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort,
+                       p.status)) {
+          ok = false;
+          break;
         }
       }
-      const float m_new = fmaxf(m, bmax);
-      const float alpha = ex2(m - m_new);
-      // pass 2: probabilities, their sum, and P (bf16) into the swizzled K-major tile
+      const float moff = m_ref * sl2;
       float sum = 0.f;
-      unsigned char* pb = smem + C::OFF_P + s * C::P_BYTES;
+      unsigned char* panel_base = smem + C::OFF_P + s * C::P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
       for (int c = 0; c < C::BN / 32; ++c) {
-        tmem_ld32(ts + c * 32, v);
-        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = (key0 + c * 32 + e <= limit) ? ex2(fmaf(v[e], sl2, -m_new)) : 0.f;
-          const float p1 = (key0 + c * 32 + e + 1 <= limit) ? ex2(fmaf(v[e + 1], sl2, -m_new)) : 0.f;
+          const float x0 = fmaf(sc[c * 32 + e], sl2, -moff);
+          const float x1 = fmaf(sc[c * 32 + e + 1], sl2, -moff);
+          const float p0 = ex2(x0);
+          const float p1 = (e & 2) ? exp2_cubic(x1) : ex2(x1);
           sum += p0 + p1;
           pk[e / 2] = pack2(p0, p1);
         }
-        unsigned char* panel = pb + (c >> 1) * C::P_PANEL + (r >> 3) * 1024 + (r & 7) * 128;
+        unsigned char* panel = panel_base + (c >> 1) * C::P_PANEL;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int chunk = ((c & 1) * 4 + k4) ^ (r & 7);
@@ -307,29 +355,34 @@ __global__ void __launch_bounds__(192, 1)
               make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
         }
       }
-      l = l * alpha + sum;
-      m = m_new;
+      l += sum;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // P visible to the MMA
-      tc_fence_before();
+      tc_fence_before();                          // and any O rescale stores ordered first
       mbar_arrive(smem_u32(&tail->p_full[s]));
-      mbar_arrive(smem_u32(&tail->s_free[s]));
-      if (j >= 1 && !correct(j - 1, alpha_prev)) {
-        ok = false;
-        break;
-      }
-      alpha_prev = alpha;
     }
-    if (ok && J > 0) ok = correct(J - 1, alpha_prev);
-    if (ok && live) {
+    if (ok && J > 0) {
+      const int i = J - 1;
+      ok = warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort, p.status);
+    }
+    if (ok) {
+      tc_fence_after();
       const float inv = 1.0f / l;
       uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)p.out +
                                             ((long long)row * p.Hq + h) * HD);
+      float v[32];
 #pragma unroll
-      for (int c = 0; c < HD / 8; ++c)
-        dst[c] = make_uint4(pack2(o[8 * c] * inv, o[8 * c + 1] * inv),
-                            pack2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                            pack2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                            pack2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+      for (int c = 0; c < HD / 32; ++c) {
+        tmem_ld32(tmem + lane_off + C::TMEM_O + c * 32, v);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8)
+            dst[c * 4 + q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                         pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                         pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                         pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+        }
+      }
     }
   }
 
