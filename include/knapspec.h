@@ -134,7 +134,8 @@ typedef struct {
   double* tpt;         /* [C][gamma_max] optional: the TPT grid */
   int32_t* best;       /* [2] required: best cell b*, best gamma* */
   double* best_tpt;    /* [1] optional: TPT(b*, gamma*) */
-  float* ref_states;   /* [n_items+1][T][d] optional: the reference states used */
+  float* ref_states;   /* [n_items+1][T][d] optional: the full model's states X^(k)
+                          the solve computed (they ride along in each item's batch) */
 } ks_result;
 
 /* Library version string (static storage). */
@@ -289,9 +290,11 @@ KS_API ks_status ks_tpt_argmax(const float* values, const double* t_draft, int32
  * a0-a6 -- the whole DP on one GPU (the spec call).
  * layers: HOST array [n_layers] of device weight pointers; cache: the full
  * model's KV cache; x0: device [T][d] fp32; ref: device [n_items+1][T][d] fp32
- * reference states, or NULL to compute them with ks_reference_forward's
- * kernels; w: HOST [n_items] item weights, or NULL to quantise t with
- * params->n_bins; t: HOST [n_items] latencies (t_Target = their sum).
+ * reference states to compare against, or NULL to use the ones the solve
+ * computes itself (X^(k) is carried as one extra state through every item's
+ * batch, with the cells' arithmetic); w: HOST [n_items] item weights, or NULL
+ * to quantise t with params->n_bins; t: HOST [n_items] latencies (t_Target =
+ * their sum).
  * The number of cells is C = sum(w) + 1; out's buffers must be sized for it
  * (ks_solve_cells() returns C).  The workspace must hold
  * ks_workspace_size(model, C, T).  Nothing is copied back to the host.

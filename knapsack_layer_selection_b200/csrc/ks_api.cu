@@ -73,35 +73,36 @@ static ks_status check_layers(const ks_model_desc* m, const ks_layer_weights* la
 
 // ---------------------------------------------------------------- workspace
 struct Workspace {
-  float *prev, *cur, *exec;   // [C][T][d] fp32
-  void *xh;                   // [C*T][d] act
-  void *q, *att;              // [C*T][qd] act
-  void *gb, *ub;              // [C*T][ffn] act
-  float* ref;                 // [n_items+1][T][d]
+  int32_t* status;            // [1] device status word of the last call (first in the buffer)
+  float *prev, *cur, *exec;   // [C+1][T][d] fp32 states: slot 0 = reference, slot b+1 = cell b
+  void *xh;                   // [C+1][T][d] act: the current item's normalised operand
+  void *q, *att;              // [(C+1)T][qd] act
+  void *gb, *ub;              // [(C+1)T][ffn] act
   uint8_t* bp;                // [n_items][C]
   float* val;                 // [C]
   double* t_draft;            // [C]
   float2* rope;               // [T][hd/2]
-  int32_t* status;            // [1]
   size_t total;
 };
 
 static size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
-static Workspace carve(const ks_model_desc* m, long long C, long long T, char* base) {
+// Lays the workspace out for batches of up to n_slots states of T tokens.
+static Workspace carve(const ks_model_desc* m, long long n_slots, long long T, char* base) {
   Workspace w{};
   const int act = m->wdtype == KS_F32 ? ACT_F32 : ACT_BF16;
   const size_t ab = act_bytes(act);
-  const long long R = C * T;
+  const long long R = n_slots * T;
   const long long d = m->d_model, qd = (long long)m->n_q_heads * m->head_dim, F = m->ffn;
   const long long n_items = 2LL * m->n_layers;
+  const long long C = n_slots;
   size_t off = 0;
   auto take = [&](size_t bytes) -> char* {
     char* p = base ? base + off : nullptr;
     off += align_up(bytes);
     return p;
   };
-  w.status = (int32_t*)take(256);   // first: the device status word of the last call
+  w.status = (int32_t*)take(256);
   w.prev = (float*)take(R * d * 4);
   w.cur = (float*)take(R * d * 4);
   w.exec = (float*)take(R * d * 4);
@@ -110,7 +111,6 @@ static Workspace carve(const ks_model_desc* m, long long C, long long T, char* b
   w.att = take(R * qd * ab);
   w.gb = take(R * F * ab);
   w.ub = take(R * F * ab);
-  w.ref = (float*)take((n_items + 1) * T * d * 4);
   w.bp = (uint8_t*)take(n_items * C);
   w.val = (float*)take(C * 4);
   w.t_draft = (double*)take(C * 8);
@@ -132,8 +132,10 @@ struct Ctx {
 };
 
 // Applies item k to E states in[0..E) -> out[0..E) (fp32 [E][T][d]).
-// The RoPE table in ws.rope must hold positions ctx .. ctx+T-1.
-static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* out) {
+// The RoPE table in ws.rope must hold positions ctx .. ctx+T-1.  With
+// xh_ready, ws.xh already holds the item's normalised operand of `in`.
+static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* out,
+                          bool xh_ready = false) {
   const ks_model_desc* m = c.m;
   const int l = k / 2;
   const ks_layer_weights& L = c.layers[l];
@@ -144,7 +146,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
   const double ab = (double)act_bytes(c.act);
   const double wb = m->wdtype == KS_F32 ? 4.0 : 2.0;
   const double Rd = (double)R;
-  {
+  if (!xh_ready) {
     ProfScope ps(KK_RMSNORM, c.st, 3.0 * Rd * d, Rd * d * (4.0 + ab));
     KS_TRY(launch_rmsnorm(in, k % 2 == 0 ? L.attn_norm : L.mlp_norm, m->wdtype, c.ws.xh, c.act, R,
                           d, m->rms_eps, c.st));
@@ -328,7 +330,8 @@ ks_status ks_workspace_size(const ks_model_desc* model, int32_t n_cells, int32_t
   KS_TRY(check_T(T));
   if (!bytes) return fail(KS_ERR_INVALID_ARG, "bytes is NULL");
   if (n_cells < 1) return fail(KS_ERR_INVALID_ARG, "n_cells must be >= 1");
-  *bytes = carve(model, n_cells, T, nullptr).total;
+  // a solve over n_cells cells keeps one more state slot (the reference)
+  *bytes = carve(model, (long long)n_cells + 1, T, nullptr).total;
   return KS_OK;
 }
 
@@ -468,7 +471,7 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   if (K + 1 > (1 << 20)) return fail(KS_ERR_UNSUPPORTED, "more than 2^20 budget cells");
   const int C = (int)(K + 1);
   Ctx c;
-  KS_TRY(make_ctx(model, layers, cache, T, C, workspace, workspace_bytes, (cudaStream_t)stream, &c));
+  KS_TRY(make_ctx(model, layers, cache, T, C + 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
   c.status = out->status;
   const cudaStream_t st = c.st;
   const long long cell = (long long)T * model->d_model;
@@ -478,21 +481,15 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     ProfScope ps(KK_ROPE_TABLE, st, 0.0, 0.0);
     KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, st));
   }
-
-  // a1: reference states X^(0..2L)
-  float* refp = out->ref_states ? out->ref_states : c.ws.ref;
-  if (ref) {
-    if (refp != ref)
-      KS_CUDA_TRY(cudaMemcpyAsync(refp, ref, (n_items + 1) * cell * sizeof(float),
-                                  cudaMemcpyDeviceToDevice, st));
-  } else {
-    KS_TRY(reference_chain(c, x0, refp));
-  }
-
-  // every cell starts from X^(0)
+  const double xb = model->wdtype == KS_F32 ? 4.0 : 2.0;
+  // Slot 0 of every state buffer carries the full model's state X^(k) through
+  // the same batched kernels as the cells, so the select target X^(k+1) comes
+  // out of each item's batch (exec slot 0) and no separate reference chain
+  // runs.  Cells start from X^(0).
   {
-    ProfScope ps(KK_BROADCAST, st, 0.0, (double)C * cell * 4.0);
-    KS_TRY(launch_broadcast(c.ws.prev, x0, C, cell, st));
+    ProfScope ps(KK_BROADCAST, st, 0.0, (double)(C + 1) * cell * (4.0 + xb));
+    KS_TRY(launch_init_states(x0, C + 1, T, model->d_model, model->rms_eps, layers[0].attn_norm,
+                              model->wdtype, c.ws.prev, c.ws.xh, out->ref_states, st));
   }
   float* prev = c.ws.prev;
   float* cur = c.ws.cur;
@@ -500,13 +497,20 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   for (int k = 0; k < n_items; ++k) {
     const int wk = ww[k];
     const int E = C - wk;
-    KS_TRY(sublayer(c, k, prev, E, c.ws.exec));
+    KS_TRY(sublayer(c, k, prev, E + 1, c.ws.exec, /*xh_ready=*/true));
     float* val = (k == n_items - 1) ? out->values : c.ws.val;
-    ProfScope ps(KK_SELECT, st, 10.0 * (2.0 * C - wk) * cell, (3.0 * C - wk) * cell * 4.0);
-    KS_TRY(launch_select(prev, c.ws.exec, refp + (long long)(k + 1) * cell, C, T,
-                         model->d_model, wk, cur, val, bp + (long long)k * C,
-                         out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
-                         out->cos_exec ? out->cos_exec + (long long)k * C : nullptr, st));
+    const void* g_next = nullptr;
+    if (k + 1 < n_items) g_next = (k + 1) % 2 == 0 ? layers[(k + 1) / 2].attn_norm
+                                                    : layers[(k + 1) / 2].mlp_norm;
+    const float* target = ref ? ref + (long long)(k + 1) * cell : nullptr;
+    ProfScope ps(KK_SELECT, st, 10.0 * (2.0 * C - wk) * cell,
+                 (3.0 * C - wk + 2.0) * cell * 4.0 + (g_next ? (C + 1.0) * cell * xb : 0.0));
+    KS_TRY(launch_select_fused(prev, c.ws.exec, target, C, T, model->d_model, wk, model->rms_eps,
+                               g_next, model->wdtype, cur, c.ws.xh, val, bp + (long long)k * C,
+                               out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
+                               out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
+                               out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr,
+                               st));
     std::swap(prev, cur);
   }
   double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;

@@ -47,6 +47,17 @@ ks_status launch_select(const float* prev, const float* exec, const float* targe
                         int d, int w, float* cur, float* val, uint8_t* bp, float* cos_s,
                         float* cos_e, cudaStream_t st);
 
+// The DP loop's select on a buffer whose slot 0 is the reference state (see
+// ks_select.cu); also writes the next item's normalised operand when g_next.
+ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
+                              int T, int d, int w, float eps, const void* g_next, int wdt,
+                              float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
+                              float* cos_e, float* ref_out, cudaStream_t st);
+
+// Slots 0..n_slots-1 of a state buffer <- x0, and their normalised operands.
+ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
+                             int wdt, float* states, void* xh, float* ref_out, cudaStream_t st);
+
 struct ItemTable {
   static constexpr int kMaxItems = 256;
   int32_t w[kMaxItems];

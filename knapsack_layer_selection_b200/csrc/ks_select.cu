@@ -96,6 +96,205 @@ ks_status launch_select(const float* prev, const float* exec, const float* targe
   return KS_OK;
 }
 
+// ---------------------------------------------------------------- fused select (DP loop)
+// Four consecutive normalised values v * sc * g[j..j+3] stored as one 8-byte
+// (bf16) or 16-byte (fp32) write.
+__device__ __forceinline__ void store_norm4(__nv_bfloat16* o, float4 v, float sc,
+                                            const __nv_bfloat16* g) {
+  const uint2 gg = *reinterpret_cast<const uint2*>(g);
+  const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&gg.x);
+  const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&gg.y);
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x * sc * __low2float(g01), v.y * sc * __high2float(g01));
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z * sc * __low2float(g23), v.w * sc * __high2float(g23));
+  uint2 out;
+  out.x = *reinterpret_cast<uint32_t*>(&a);
+  out.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(o) = out;
+}
+
+__device__ __forceinline__ void store_norm4(float* o, float4 v, float sc, const float* g) {
+  const float4 gg = *reinterpret_cast<const float4*>(g);
+  *reinterpret_cast<float4*>(o) = make_float4(v.x * sc * gg.x, v.y * sc * gg.y, v.z * sc * gg.z,
+                                              v.w * sc * gg.w);
+}
+
+// The DP loop's select step on a state buffer with a leading reference slot:
+// slot 0 holds the full model's state X^(k), slots 1..C the cells 0..C-1.  The
+// batched forward of item k ran on slots 0..E (E = C - w), so exec slot 0 is
+// X^(k+1) and exec slot e+1 is the execute candidate of cell e + w.
+//   block 0     : the reference slot -- cur[0] = exec[0];
+//   block b + 1 : cell b -- the select of select_kernel against the target
+//                 (the caller's X^(k+1), or exec slot 0).
+// Every block also writes the next item's normalised operand of the state it
+// stores, x^ = x / sqrt(mean_t(x^2) + eps) * g_next, from the per-token sums of
+// squares the cosine already needs (fp64), so no separate RMSNorm pass runs.
+// A slot's arithmetic does not depend on its position, so the all-execute cell
+// and the reference slot stay bit-identical.
+template <typename TX, typename TG>
+__global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
+    const float* __restrict__ prev, const float* __restrict__ exec,
+    const float* __restrict__ target_in, int T, int d, int w, float eps,
+    const TG* __restrict__ g_next, float* __restrict__ cur, TX* __restrict__ xh_next,
+    float* __restrict__ val, uint8_t* __restrict__ bp, float* __restrict__ cos_s_out,
+    float* __restrict__ cos_e_out, float* __restrict__ ref_out) {
+  __shared__ double cs_tok[kSelectMaxT];
+  __shared__ double ce_tok[kSelectMaxT];
+  __shared__ float inv_s[kSelectMaxT];
+  __shared__ float inv_e[kSelectMaxT];
+  __shared__ int take_sh;
+  const long long cell = (long long)T * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_warps = blockDim.x >> 5;
+  const int d4 = d / 4;
+  const bool is_ref = blockIdx.x == 0;
+  const int b = (int)blockIdx.x - 1;
+  const bool has_e = !is_ref && b >= w;
+  // "s" is the skip candidate (or, for the reference slot, the state to keep)
+  const float* s_base = is_ref ? exec : prev + (long long)(b + 1) * cell;
+  const float* e_base = has_e ? exec + (long long)(b - w + 1) * cell : nullptr;
+  const float* target = target_in ? target_in : exec;
+  for (int t = warp; t < T; t += n_warps) {
+    const float4* s4 = (const float4*)(s_base + (long long)t * d);
+    const float4* r4 = (const float4*)(target + (long long)t * d);
+    const float4* e4 = has_e ? (const float4*)(e_base + (long long)t * d) : nullptr;
+    double sr = 0, ss = 0, rr = 0, er = 0, ee = 0;
+    for (int i = lane; i < d4; i += 32) {
+      const float4 sv = s4[i];
+      ss += (double)sv.x * sv.x + (double)sv.y * sv.y + (double)sv.z * sv.z + (double)sv.w * sv.w;
+      if (!is_ref) {
+        const float4 r = r4[i];
+        sr += (double)sv.x * r.x + (double)sv.y * r.y + (double)sv.z * r.z + (double)sv.w * r.w;
+        rr += (double)r.x * r.x + (double)r.y * r.y + (double)r.z * r.z + (double)r.w * r.w;
+        if (has_e) {
+          const float4 e = e4[i];
+          er += (double)e.x * r.x + (double)e.y * r.y + (double)e.z * r.z + (double)e.w * r.w;
+          ee += (double)e.x * e.x + (double)e.y * e.y + (double)e.z * e.z + (double)e.w * e.w;
+        }
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      sr += __shfl_xor_sync(0xffffffffu, sr, o);
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      rr += __shfl_xor_sync(0xffffffffu, rr, o);
+      er += __shfl_xor_sync(0xffffffffu, er, o);
+      ee += __shfl_xor_sync(0xffffffffu, ee, o);
+    }
+    if (lane == 0) {
+      cs_tok[t] = is_ref ? 0.0 : sr / sqrt(ss * rr);
+      ce_tok[t] = has_e ? er / sqrt(ee * rr) : 0.0;
+      inv_s[t] = (float)(1.0 / sqrt(ss / (double)d + (double)eps));
+      inv_e[t] = (float)(1.0 / sqrt(ee / (double)d + (double)eps));
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int take = 0;
+    if (!is_ref) {
+      double ms = 0.0, me = 0.0;
+      for (int t = 0; t < T; ++t) {
+        ms += cs_tok[t];
+        me += ce_tok[t];
+      }
+      ms /= (double)T;
+      me /= (double)T;
+      take = (has_e && me > ms) ? 1 : 0;
+      val[b] = (float)(take ? me : ms);
+      bp[b] = (uint8_t)take;
+      if (cos_s_out) cos_s_out[b] = (float)ms;
+      if (cos_e_out) cos_e_out[b] = has_e ? (float)me : __int_as_float(0x7fc00000);
+    }
+    take_sh = take;
+  }
+  __syncthreads();
+  const bool take = take_sh != 0;
+  const float4* src = (const float4*)(take ? e_base : s_base);
+  const float* inv = take ? inv_e : inv_s;
+  const long long slot = is_ref ? 0 : (long long)(b + 1);
+  float4* dst = (float4*)(cur + slot * cell);
+  float4* rdst = (is_ref && ref_out) ? (float4*)ref_out : nullptr;
+  TX* xdst = g_next ? xh_next + slot * cell : nullptr;
+  const long long n4 = cell / 4;
+  for (long long i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = v;
+    if (rdst) rdst[i] = v;
+    if (xdst) {
+      const int t = (int)(i / d4);
+      const int j = (int)(i - (long long)t * d4) * 4;
+      store_norm4(xdst + i * 4, v, inv[t], g_next + j);
+    }
+  }
+}
+
+ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
+                              int T, int d, int w, float eps, const void* g_next, int wdt,
+                              float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
+                              float* cos_e, float* ref_out, cudaStream_t st) {
+  if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "select: T above 256");
+  if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "select: d must be a multiple of 4");
+  if (wdt == KS_BF16)
+    select_fused_kernel<__nv_bfloat16, __nv_bfloat16><<<C + 1, kSelectThreads, 0, st>>>(
+        prev, exec, target, T, d, w, eps, (const __nv_bfloat16*)g_next, cur,
+        (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out);
+  else
+    select_fused_kernel<float, float><<<C + 1, kSelectThreads, 0, st>>>(
+        prev, exec, target, T, d, w, eps, (const float*)g_next, cur, (float*)xh_next, val, bp,
+        cos_s, cos_e, ref_out);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+// Fills slots 0..C of the state buffer with x0 and the first item's operand
+// x^ = x0 / sqrt(mean(x0^2) + eps) * g (the same sums and formula as the fused
+// select, so slot contents match what a select would have written).
+template <typename TX, typename TG>
+__global__ void __launch_bounds__(kSelectThreads) init_states_kernel(
+    const float* __restrict__ x0, int T, int d, float eps, const TG* __restrict__ g,
+    float* __restrict__ states, TX* __restrict__ xh, float* __restrict__ ref_out) {
+  __shared__ float inv_s[kSelectMaxT];
+  const long long cell = (long long)T * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d4 = d / 4;
+  for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) {
+    const float4* s4 = (const float4*)(x0 + (long long)t * d);
+    double ss = 0;
+    for (int i = lane; i < d4; i += 32) {
+      const float4 sv = s4[i];
+      ss += (double)sv.x * sv.x + (double)sv.y * sv.y + (double)sv.z * sv.z + (double)sv.w * sv.w;
+    }
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) inv_s[t] = (float)(1.0 / sqrt(ss / (double)d + (double)eps));
+  }
+  __syncthreads();
+  const long long slot = blockIdx.x;
+  const float4* src = (const float4*)x0;
+  float4* dst = (float4*)(states + slot * cell);
+  float4* rdst = (slot == 0 && ref_out) ? (float4*)ref_out : nullptr;
+  TX* xdst = xh + slot * cell;
+  for (long long i = threadIdx.x; i < cell / 4; i += blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = v;
+    if (rdst) rdst[i] = v;
+    const int t = (int)(i / d4);
+    const int j = (int)(i - (long long)t * d4) * 4;
+    store_norm4(xdst + i * 4, v, inv_s[t], g + j);
+  }
+}
+
+ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
+                             int wdt, float* states, void* xh, float* ref_out, cudaStream_t st) {
+  if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "init: T above 256");
+  if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "init: d must be a multiple of 4");
+  if (wdt == KS_BF16)
+    init_states_kernel<__nv_bfloat16, __nv_bfloat16><<<n_slots, kSelectThreads, 0, st>>>(
+        x0, T, d, eps, (const __nv_bfloat16*)g, states, (__nv_bfloat16*)xh, ref_out);
+  else
+    init_states_kernel<float, float><<<n_slots, kSelectThreads, 0, st>>>(
+        x0, T, d, eps, (const float*)g, states, (float*)xh, ref_out);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
 // ---------------------------------------------------------------- reconstruct
 constexpr int kMaxWords = ItemTable::kMaxItems / 64;
 
