@@ -310,6 +310,18 @@ KS_API ks_status ks_solve_cells(int32_t n_items, const int32_t* w, const double*
                          const ks_params* params, int32_t* n_cells);
 
 /*
+ * Diagnostics of the device-side failure handling (the paper has no
+ * counterpart).  Launches one kernel whose mbarrier wait nothing completes,
+ * bounded by the routine every tensor-core kernel's waits use, with a limit of
+ * limit_us microseconds (1 .. 2,000,000).  When the bound works the kernel
+ * returns on its own and writes KS_ERR_TIMEOUT into *status (device int32,
+ * which the caller zeroes first) and the nanoseconds it waited into *waited_ns
+ * (device uint64, or NULL); the CUDA context stays usable.
+ */
+KS_API ks_status ks_check_bounded_wait(uint32_t limit_us, int32_t* status, uint64_t* waited_ns,
+                                       ks_stream_t stream);
+
+/*
  * Launch accounting.  Between ks_profile_start and ks_profile_stop the library
  * counts the kernels it enqueues per kind, adds up their algorithmic FLOPs and
  * bytes (the work the DP defines, not what the hardware moved) and, when

@@ -64,7 +64,8 @@ EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weigh
            "ks_workspace_size", "ks_sublayer_forward", "ks_reference_forward",
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
            "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
-           "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16"]
+           "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16",
+           "ks_check_bounded_wait"]
 
 _lib = None
 
@@ -96,6 +97,7 @@ def load() -> ctypes.CDLL:
         "ks_reference_forward_noalloc": ([P, P, P, I32, P, P, P], ctypes.c_int),
         "ks_workspace_status": ([P, ctypes.POINTER(I32), P], ctypes.c_int),
         "ks_gemm_bf16": ([P, P, P, P, I32, I32, I32, P, P], ctypes.c_int),
+        "ks_check_bounded_wait": ([ctypes.c_uint32, P, P, P], ctypes.c_int),
         "ks_attention_bf16": ([P, P, P, I64, I32, I32, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
     }
@@ -234,6 +236,13 @@ def attention_bf16(q: torch.Tensor, k_layer: torch.Tensor, v_layer: torch.Tensor
                                     _dev(v_layer, torch.bfloat16, "v"), rows, R, T, Hq, Hkv, hd,
                                     ctx, _dev(out, torch.bfloat16, "out"),
                                     _dev(status, torch.int32, "status"), _stream()))
+
+
+def check_bounded_wait(limit_us: int, status: torch.Tensor,
+                       waited_ns: Optional[torch.Tensor] = None) -> None:
+    """Run one device wait that nothing completes, bounded to limit_us."""
+    _check(load().ks_check_bounded_wait(limit_us, _dev(status, torch.int32, "status"),
+                                        _dev(waited_ns, torch.int64, "waited_ns"), _stream()))
 
 
 def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:
