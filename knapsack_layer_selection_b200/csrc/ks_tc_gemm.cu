@@ -14,8 +14,9 @@
 //   warps 2-5 -- epilogue: tcgen05.ld 32 columns at a time from their 32-lane
 //              quarter, apply the fused epilogue, store to global memory.
 // The accumulator double buffer lets the epilogue of tile i overlap the MMAs of
-// tile i+1.  Tiles are walked M-fastest so CTAs running together share one
-// weight tile through L2.  No split-K: every output is the same fixed-order
+// tile i+1.  Tiles are walked in groups of m-tiles (m fastest inside a group):
+// the CTAs running together share a few weight tiles through L2, and a group's
+// activation rows stay resident while its weight columns stream.  No split-K: every output is the same fixed-order
 // sum over K whatever M is, so a row's result does not depend on its batch.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -72,8 +73,22 @@ struct GemmParams {
   int32_t* status;
   int M, N_out, K;
   int tiles_m, tiles_n;
+  int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
   int T, head_dim;
 };
+
+// Tile t of the walk -> (m-tile, n-tile).  Tiles go in groups of group_m m-tiles;
+// inside a group the m index runs fastest, so the CTAs in flight share a few
+// weight tiles and the group's A rows stay in L2 while its weight columns stream.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
+  const int per_group = p.group_m * p.tiles_n;
+  const int g = t / per_group;
+  const int local = t - g * per_group;
+  const int m_base = g * p.group_m;
+  const int rows = min(p.group_m, p.tiles_m - m_base);
+  tm = m_base + local % rows;
+  tn = local / rows;
+}
 
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -120,8 +135,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int m0 = (t % p.tiles_m) * BM;
-        const int tn = t / p.tiles_m;
+        int tm, tn;
+        tile_coords(p, t, tm, tn);
+        const int m0 = tm * BM;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t r = (uint32_t)(it / STAGES);
@@ -191,8 +207,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got = mbar_wait(smem_u32(&tail->tfull[acc]), ar & 1u, abort, p.status);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int m0 = (t % p.tiles_m) * BM;
-      const int tn = t / p.tiles_m;
+      int tm, tn;
+      tile_coords(p, t, tm, tn);
+      const int m0 = tm * BM;
       const int row = m0 + q * 32 + lane;
       const bool live = row < p.M;
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
@@ -372,6 +389,15 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
   gp.K = K;
   gp.tiles_m = (M + BM - 1) / BM;
   gp.tiles_n = N / bn_out;
+  // a group's A rows (group_m x 128 rows x K) should stay well inside one die's
+  // half of L2 (~32 MB) while the weight columns stream past them
+  {
+    const long long a_tile = (long long)BM * K * 2;
+    long long g = (32ll << 20) / a_tile;
+    if (g < 8) g = 8;
+    if (g > 32) g = 32;
+    gp.group_m = (int)(g < gp.tiles_m ? g : gp.tiles_m);
+  }
   gp.T = T;
   gp.head_dim = head_dim;
   switch (epi) {
