@@ -25,8 +25,8 @@
 //                relative to a reference maximum that moves only when the row's
 //                maximum grows by more than 2^8, and only then is the row's O in
 //                TMEM rescaled (after the previous P.V has landed).  exp2 runs
-//                on the MUFU unit for three of every four scores and as a cubic
-//                on the FMA pipe for the fourth.  Only blocks that reach past
+//                on the MUFU unit for five of every eight scores and as a cubic
+//                on the FMA/integer pipes for the other three.  Only blocks that reach past
 //                position ctx are masked.  P goes to shared memory as bf16 in the
 //                swizzled K-major layout the MMA reads; O is normalised by the
 //                running sum once, at the end.
@@ -116,22 +116,25 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of arguments as 2^floor(x) * q(x - floor(x)), q a cubic fitted
-// to 2^f on [0, 1) for minimal relative error (7.5e-5, far below the bf16
-// rounding of P); the polynomial steps run two-wide on the FMA pipe.  Used for
-// a share of the scores so the MUFU unit is not the only source of exp2.
+// 2^x for a pair of arguments as 2^n * q(x - n) with n = round(x): adding
+// 1.5 * 2^23 leaves n in the low mantissa bits (and, shifted by 23, exactly the
+// exponent increment), so no conversion instruction is needed; q is a cubic
+// fitted to 2^f on [-1/2, 1/2] for minimal relative error (7.5e-5, far below
+// the bf16 rounding of P).  Every step runs on the FMA or integer pipes, two
+// lanes per f32x2 instruction, which takes load off the MUFU unit.
 __device__ __forceinline__ void exp2_cubic2(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const float f0 = floorf(x0), f1 = floorf(x1);
-  const uint64_t f = add2(pk2(x0, x1), pk2(-f0, -f1));
-  uint64_t q = fma2(pk2(0.07802403f, 0.07802403f), f, pk2(0.22606707f, 0.22606707f));
-  q = fma2(q, f, pk2(0.69583398f, 0.69583398f));
-  q = fma2(q, f, pk2(0.99992514f, 0.99992514f));
-  float q0, q1;
+  const uint64_t x = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));   // results stay normal
+  const uint64_t t = add2(x, pk2(12582912.0f, 12582912.0f));
+  const uint64_t n = add2(t, pk2(-12582912.0f, -12582912.0f));     // round(x) as a float
+  const uint64_t f = fma2(n, pk2(-1.0f, -1.0f), x);                // x - round(x)
+  uint64_t q = fma2(pk2(0.055171434f, 0.055171434f), f, pk2(0.24261081f, 0.24261081f));
+  q = fma2(q, f, pk2(0.69326097f, 0.69326097f));
+  q = fma2(q, f, pk2(0.99992812f, 0.99992812f));
+  float q0, q1, t0, t1;
   upk2(q, q0, q1);
-  y0 = __int_as_float(__float_as_int(q0) + ((int)f0 << 23));
-  y1 = __int_as_float(__float_as_int(q1) + ((int)f1 << 23));
+  upk2(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // 32 consecutive fp32 columns into this thread's TMEM lane (32x32b shape, x32).
@@ -442,8 +445,8 @@ __global__ void __launch_bounds__(320, 1)
           const int k = c8 * 8 + e;
           float x0, x1, p0, p1;
           upk2(fma2(pk2(sc[k], sc[k + 1]), scale2, moff2), x0, x1);
-          if (e == 6) {
-            exp2_cubic2(x0, x1, p0, p1);           // one pair in four on the FMA pipe
+          if ((c8 & 1) ? (e == 2 || e == 6) : (e == 6)) {
+            exp2_cubic2(x0, x1, p0, p1);           // three pairs in eight on the FMA pipe
           } else {
             p0 = ex2(x0);
             p1 = ex2(x1);
