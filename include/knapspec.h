@@ -109,12 +109,21 @@ typedef struct {
   int32_t ctx;
 } ks_cache_desc;
 
+/* Budget semantics of a cell b (the review notes the paper's main text and
+ * appendix initialise the table differently, referee major 1). */
+typedef enum {
+  KS_BUDGET_AT_MOST = 0,   /* b caps the used weight; every cell starts from X^(0) */
+  KS_BUDGET_EXACT = 1      /* b is the used weight exactly; only cell 0 starts valid, a
+                              cell no subset fills stays invalid (value NaN) */
+} ks_budget_mode;
+
 /* Selection parameters.  alpha(b) = clamp((value_b - alpha_lo) / alpha_scale,
  * 0, alpha_max) is the acceptance-rate stand-in; gamma runs 1 .. gamma_max. */
 typedef struct {
   int32_t gamma_max;
   int32_t n_bins;      /* budget-grid bins for ks_quantize_weights (ks_solve
                           uses it when no weights are passed) */
+  int32_t budget_mode; /* ks_budget_mode */
   double alpha_lo;
   double alpha_scale;
   double alpha_max;
@@ -126,8 +135,8 @@ typedef struct {
   int32_t* status;     /* [1] required: 0, or a ks_status a kernel wrote */
   float* values;       /* [C] required: final-row value of every cell */
   uint64_t* sets;      /* [C][words] required: bit k set = item k executed */
-  int32_t* used_w;     /* [C] optional: sum of the executed items' weights */
-  double* t_draft;     /* [C] optional: sum of the executed items' latencies */
+  int32_t* used_w;     /* [C] optional: sum of the executed items' weights (-1: invalid cell) */
+  double* t_draft;     /* [C] optional: sum of the executed items' latencies (NaN: invalid) */
   uint8_t* bp;         /* [n_items][C] optional: 1 = execute won */
   float* cos_skip;     /* [n_items][C] optional: skip candidate's value */
   float* cos_exec;     /* [n_items][C] optional: execute candidate's value (NaN if b < w) */

@@ -42,8 +42,12 @@ class CacheDesc(ctypes.Structure):
                 ("cache_rows", ctypes.c_int64), ("ctx", ctypes.c_int32)]
 
 
+KS_BUDGET_AT_MOST, KS_BUDGET_EXACT = 0, 1
+
+
 class Params(ctypes.Structure):
     _fields_ = [("gamma_max", ctypes.c_int32), ("n_bins", ctypes.c_int32),
+                ("budget_mode", ctypes.c_int32),
                 ("alpha_lo", ctypes.c_double), ("alpha_scale", ctypes.c_double),
                 ("alpha_max", ctypes.c_double)]
 
@@ -159,8 +163,9 @@ def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int) -> CacheD
 
 
 def params(gamma_max: int, n_bins: int = 0, alpha_lo: float = 0.5, alpha_scale: float = 0.5,
-           alpha_max: float = 0.99) -> Params:
-    return Params(gamma_max, n_bins, alpha_lo, alpha_scale, alpha_max)
+           alpha_max: float = 0.99, budget_mode: str = "at_most") -> Params:
+    mode = {"at_most": KS_BUDGET_AT_MOST, "exact": KS_BUDGET_EXACT}[budget_mode]
+    return Params(gamma_max, n_bins, mode, alpha_lo, alpha_scale, alpha_max)
 
 
 # ---------------------------------------------------------------- calls

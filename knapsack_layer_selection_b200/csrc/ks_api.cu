@@ -79,6 +79,7 @@ struct Workspace {
   void *q, *att;              // [(C+1)T][qd] act
   void *gb, *ub;              // [(C+1)T][ffn] act
   uint8_t* bp;                // [n_items][C]
+  uint8_t *valid_a, *valid_b; // [C] exact-budget validity, ping-pong
   float* val;                 // [C]
   double* t_draft;            // [C]
   float2* rope;               // [T][hd/2]
@@ -112,6 +113,8 @@ static Workspace carve(const ks_model_desc* m, long long n_slots, long long T, c
   w.gb = take(R * F * ab);
   w.ub = take(R * F * ab);
   w.bp = (uint8_t*)take(n_items * C);
+  w.valid_a = (uint8_t*)take(C);
+  w.valid_b = (uint8_t*)take(C);
   w.val = (float*)take(C * 4);
   w.t_draft = (double*)take(C * 8);
   w.rope = (float2*)take(T * (m->head_dim / 2) * sizeof(float2));
@@ -404,7 +407,7 @@ ks_status ks_reconstruct(const uint8_t* bp, const int32_t* w, const double* t, i
   if (n_items < 1 || n_items > ItemTable::kMaxItems || C < 1)
     return fail(KS_ERR_INVALID_ARG, "reconstruct: n_items in 1..256, C >= 1");
   return launch_reconstruct(bp, w, t, nullptr, n_items, C, sets, used_w, t_draft, status,
-                            (cudaStream_t)stream);
+                            nullptr, (cudaStream_t)stream);
 }
 
 ks_status ks_tpt_argmax(const float* values, const double* t_draft, int32_t C, double t_target,
@@ -455,6 +458,8 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     return fail(KS_ERR_INVALID_ARG, "solve: result needs status, values, sets and best");
   if (params->gamma_max < 1 || !(params->alpha_scale > 0.0))
     return fail(KS_ERR_INVALID_ARG, "solve: gamma_max >= 1 and alpha_scale > 0");
+  if (params->budget_mode != KS_BUDGET_AT_MOST && params->budget_mode != KS_BUDGET_EXACT)
+    return fail(KS_ERR_INVALID_ARG, "solve: budget_mode must be KS_BUDGET_AT_MOST or KS_BUDGET_EXACT");
   const int n_items = 2 * model->n_layers;
   std::vector<int32_t> ww;
   KS_TRY(resolve_weights(n_items, w, t, params, &ww));
@@ -494,6 +499,10 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   float* prev = c.ws.prev;
   float* cur = c.ws.cur;
   uint8_t* bp = out->bp ? out->bp : c.ws.bp;
+  const bool exact = params->budget_mode == KS_BUDGET_EXACT;
+  uint8_t* vprev = exact ? c.ws.valid_a : nullptr;
+  uint8_t* vcur = exact ? c.ws.valid_b : nullptr;
+  if (exact) KS_TRY(launch_init_valid(vprev, C, st));
   for (int k = 0; k < n_items; ++k) {
     const int wk = ww[k];
     const int E = C - wk;
@@ -510,14 +519,15 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
                                out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
                                out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
                                out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr,
-                               st));
+                               vprev, vcur, st));
     std::swap(prev, cur);
+    std::swap(vprev, vcur);
   }
   double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;
   {
     ProfScope ps(KK_RECONSTRUCT, st, 0.0, (double)n_items * C);
     KS_TRY(launch_reconstruct(bp, nullptr, nullptr, &tab, n_items, C, out->sets, out->used_w, tdp,
-                              out->status, st));
+                              out->status, vprev, st));
   }
   ProfScope ps(KK_TPT, st, 0.0, (double)C * 12.0);
   KS_TRY(launch_tpt(out->values, tdp, C, t_target, params->gamma_max, params->alpha_lo,

@@ -49,10 +49,13 @@ ks_status launch_select(const float* prev, const float* exec, const float* targe
 
 // The DP loop's select on a buffer whose slot 0 is the reference state (see
 // ks_select.cu); also writes the next item's normalised operand when g_next.
+// valid_prev / valid_cur (both NULL: every cell valid) carry the exact-budget
+// validity of the cells from row to row.
 ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
-                              float* cos_e, float* ref_out, cudaStream_t st);
+                              float* cos_e, float* ref_out, const uint8_t* valid_prev,
+                              uint8_t* valid_cur, cudaStream_t st);
 
 // Slots 0..n_slots-1 of a state buffer <- x0, and their normalised operands.
 ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
@@ -64,9 +67,14 @@ struct ItemTable {
   double t[kMaxItems];
 };
 
+// valid (NULL: all valid): invalid cells get an empty set, used weight -1, NaN t_draft.
 ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* t,
                              const ItemTable* tab, int n_items, int C, uint64_t* sets,
-                             int32_t* used_w, double* t_draft, int32_t* status, cudaStream_t st);
+                             int32_t* used_w, double* t_draft, int32_t* status,
+                             const uint8_t* valid, cudaStream_t st);
+
+// valid[b] = (b == 0) for the exact-budget mode.
+ks_status launch_init_valid(uint8_t* valid, int C, cudaStream_t st);
 
 ks_status launch_tpt(const float* values, const double* t_draft, int C, double t_target,
                      int gamma_max, double lo, double scale, double amax, double* tpt,

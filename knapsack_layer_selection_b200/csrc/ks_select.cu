@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
     const float* __restrict__ target_in, int T, int d, int w, float eps,
     const TG* __restrict__ g_next, float* __restrict__ cur, TX* __restrict__ xh_next,
     float* __restrict__ val, uint8_t* __restrict__ bp, float* __restrict__ cos_s_out,
-    float* __restrict__ cos_e_out, float* __restrict__ ref_out) {
+    float* __restrict__ cos_e_out, float* __restrict__ ref_out,
+    const uint8_t* __restrict__ valid_prev, uint8_t* __restrict__ valid_cur) {
   __shared__ double cs_tok[kSelectMaxT];
   __shared__ double ce_tok[kSelectMaxT];
   __shared__ float inv_s[kSelectMaxT];
@@ -197,11 +198,16 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
       }
       ms /= (double)T;
       me /= (double)T;
-      take = (has_e && me > ms) ? 1 : 0;
-      val[b] = (float)(take ? me : ms);
+      // exact-budget mode: a candidate exists only if its source cell is valid
+      const bool sv = valid_prev ? valid_prev[b] != 0 : true;
+      const bool ev = has_e && (valid_prev ? valid_prev[b - w] != 0 : true);
+      take = ev && (!sv || me > ms) ? 1 : 0;
+      const float nan = __int_as_float(0x7fc00000);
+      val[b] = (sv || ev) ? (float)(take ? me : ms) : nan;
       bp[b] = (uint8_t)take;
-      if (cos_s_out) cos_s_out[b] = (float)ms;
-      if (cos_e_out) cos_e_out[b] = has_e ? (float)me : __int_as_float(0x7fc00000);
+      if (valid_cur) valid_cur[b] = (uint8_t)(sv || ev);
+      if (cos_s_out) cos_s_out[b] = sv ? (float)ms : nan;
+      if (cos_e_out) cos_e_out[b] = ev ? (float)me : nan;
     }
     take_sh = take;
   }
@@ -229,17 +235,18 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
 ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
-                              float* cos_e, float* ref_out, cudaStream_t st) {
+                              float* cos_e, float* ref_out, const uint8_t* valid_prev,
+                              uint8_t* valid_cur, cudaStream_t st) {
   if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "select: T above 256");
   if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "select: d must be a multiple of 4");
   if (wdt == KS_BF16)
     select_fused_kernel<__nv_bfloat16, __nv_bfloat16><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const __nv_bfloat16*)g_next, cur,
-        (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out);
+        (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out, valid_prev, valid_cur);
   else
     select_fused_kernel<float, float><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const float*)g_next, cur, (float*)xh_next, val, bp,
-        cos_s, cos_e, ref_out);
+        cos_s, cos_e, ref_out, valid_prev, valid_cur);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -302,10 +309,16 @@ __global__ void reconstruct_kernel(const uint8_t* __restrict__ bp, const int32_t
                                    const double* __restrict__ t_dev, ItemTable tab, bool use_tab,
                                    int n_items, int C, uint64_t* __restrict__ sets,
                                    int32_t* __restrict__ used_w, double* __restrict__ t_draft,
-                                   int32_t* status) {
+                                   int32_t* status, const uint8_t* __restrict__ valid) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= C) return;
   const int words = (n_items + 63) / 64;
+  if (valid && !valid[b]) {   // no subset fills this exact budget
+    for (int i = 0; i < words; ++i) sets[(long long)b * words + i] = 0;
+    if (used_w) used_w[b] = -1;
+    if (t_draft) t_draft[b] = __longlong_as_double(0x7ff8000000000000ll);
+    return;
+  }
   uint64_t bits[kMaxWords];
 #pragma unroll
   for (int i = 0; i < kMaxWords; ++i) bits[i] = 0;
@@ -333,12 +346,24 @@ __global__ void reconstruct_kernel(const uint8_t* __restrict__ bp, const int32_t
 
 ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* t,
                              const ItemTable* tab, int n_items, int C, uint64_t* sets,
-                             int32_t* used_w, double* t_draft, int32_t* status, cudaStream_t st) {
+                             int32_t* used_w, double* t_draft, int32_t* status,
+                             const uint8_t* valid, cudaStream_t st) {
   if (n_items > ItemTable::kMaxItems) return fail(KS_ERR_UNSUPPORTED, "reconstruct: > 256 items");
   ItemTable empty;
   const ItemTable& tb = tab ? *tab : empty;
   reconstruct_kernel<<<ceil_div(C, 128), 128, 0, st>>>(bp, w, t, tb, tab != nullptr, n_items, C,
-                                                       sets, used_w, t_draft, status);
+                                                       sets, used_w, t_draft, status, valid);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+__global__ void init_valid_kernel(uint8_t* valid, int C) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < C) valid[b] = (uint8_t)(b == 0);
+}
+
+ks_status launch_init_valid(uint8_t* valid, int C, cudaStream_t st) {
+  init_valid_kernel<<<ceil_div(C, 256), 256, 0, st>>>(valid, C);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }

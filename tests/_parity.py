@@ -72,11 +72,19 @@ def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=Non
     r.bp_mismatch_untainted = int(((bp_o != bp_g) & ~taint).sum())
     # values: final row always, every row when the GPU exported them
     ok = ~taint[-1]
-    err = np.abs(gpu["values"].astype(np.float64) - orc.values)
+
+    def errors(g, o):
+        # invalid cells (exact-budget mode) are NaN on both sides; NaN on one side only fails
+        g = g.astype(np.float64)
+        both = np.isnan(g) & np.isnan(o)
+        e = np.where(both, 0.0, np.abs(g - o))
+        return np.where(np.isnan(e), np.inf, e)
+
+    err = errors(gpu["values"], orc.values)
     r.val_max_err = float(np.max(err[ok])) if ok.any() else 0.0
     r.val_fail = int(np.sum(err[ok] > val_tol))
     if rows_val_gpu is not None:
-        e2 = np.abs(rows_val_gpu.astype(np.float64) - orc.dp.val[1:])
+        e2 = errors(rows_val_gpu, orc.dp.val[1:])
         m = ~taint
         r.val_max_err = max(r.val_max_err, float(np.max(e2[m])) if m.any() else 0.0)
         r.val_fail += int(np.sum(e2[m] > val_tol))

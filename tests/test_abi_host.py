@@ -135,6 +135,17 @@ def test_solve_rejects_null_and_short_workspace_before_any_launch(lib):
     assert st == 1 and b"cache_rows" in lib.ks_last_error()
 
 
+def test_solve_rejects_unknown_budget_mode(lib):
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    prm = B.params(4, 8)
+    prm.budget_mode = 7
+    t = (ctypes.c_double * 2)(1.0, 1.0)
+    res = B.Result(*([256] * 12))
+    st = lib.ks_solve(ctypes.byref(m), None, None, 4, ctypes.c_void_p(256), None, None, t,
+                      ctypes.byref(prm), None, 0, ctypes.byref(res), None)
+    assert st == 1 and b"budget_mode" in lib.ks_last_error()
+
+
 def test_step_calls_reject_bad_arguments(lib):
     st = lib.ks_select_step(None, None, None, 4, 4, 64, 1, None, None, None, None, None, None)
     assert st == 1

@@ -28,11 +28,11 @@ def lib():
     return B.load()
 
 
-def make_solver(wl, inp_gpu, w=None, t=None, keep_cos=True):
+def make_solver(wl, inp_gpu, w=None, t=None, keep_cos=True, mode="at_most"):
     m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
                      wl.rms_eps, wl.rope_base, wl.wdtype)
     t = wl.latencies() if t is None else t
-    prm = B.params(wl.gamma_max, wl.n_bins)
+    prm = B.params(wl.gamma_max, wl.n_bins, budget_mode=mode)
     return B.Solver(m, inp_gpu.layers, inp_gpu.k_cache, inp_gpu.v_cache, wl.ctx, wl.T, t, prm,
                     w=w, keep_cos=keep_cos)
 
@@ -53,8 +53,8 @@ def gpu_result(solver):
 _cache = {}
 
 
-def solved(name, n_layers=None):
-    key = (name, n_layers)
+def solved(name, n_layers=None, mode="at_most"):
+    key = (name, n_layers, mode)
     if key in _cache:
         return _cache[key]
     wl = W.WORKLOADS[name]
@@ -66,11 +66,11 @@ def solved(name, n_layers=None):
         wl = inp.wl
         t, w = t[:2 * n_layers], w[:2 * n_layers]
     g = inp.to("cuda")
-    solver = make_solver(wl, g, w=w, t=t)
+    solver = make_solver(wl, g, w=w, t=t, mode=mode)
     solver.solve(g.x0)
     res = gpu_result(solver)
     orc = O.dp_solve(oracle_model(inp), x0_np(inp), wl.ctx, w, t, wl.gamma_max,
-                     per_cell=(wl.wdtype == "f32"))
+                     per_cell=(wl.wdtype == "f32"), mode=mode)
     _cache[key] = (wl, inp, g, solver, res, orc, w, t)
     return _cache[key]
 
@@ -90,6 +90,26 @@ def test_solve_matches_oracle(name, n_layers):
     for b in range(C):
         assert res["used_w"][b] <= b
         assert res["used_w"][b] == sum(w[k] for k in res["sets"][b])
+
+
+@pytest.mark.parametrize("name,n_layers", [("tiny", None), ("small", 4), ("small", None)])
+def test_exact_budget_mode_matches_oracle(name, n_layers):
+    """The paper's exact-budget table (only g[0,0] starts valid): validity is
+    integer logic and must match exactly; values and choices under the same
+    near-tie/taint rule as the at-most mode."""
+    wl, inp, g, solver, res, orc, w, t = solved(name, n_layers, "exact")
+    rep = compare_solve(orc, res, w, VAL_TOL[wl.wdtype], wl.n_items, rows_val_gpu=res["rows"])
+    print(f"\n{name}/{n_layers} exact: {rep}")
+    rep.assert_ok()
+    valid_o = orc.dp.valid[-1]
+    assert np.array_equal(np.isfinite(res["values"]), valid_o)
+    for b in range(len(valid_o)):
+        if valid_o[b]:
+            assert res["used_w"][b] == b
+        else:
+            assert res["used_w"][b] == -1 and res["sets"][b] == []
+    # reachable budgets are exactly the subset sums
+    assert abs(res["values"][-1] - 1.0) <= 1e-6
 
 
 def test_small_first_8_items_bounded_by_exhaustive_search():
