@@ -127,6 +127,13 @@ typedef struct {
   double alpha_lo;
   double alpha_scale;
   double alpha_max;
+  /* Optional pruning (review: tau = 0.5 cosine threshold, K/2 skipped-weight
+   * cap; "Assumptions & free parameters", "Reading between the lines").  After
+   * item k a cell is dropped (invalid: value NaN, never read again, no set) if
+   * its kept value is below prune_tau, or if its budget b < W_k - skip_cap with
+   * W_k = w_0 + .. + w_k.  prune_tau = -INFINITY and skip_cap < 0 turn them off. */
+  double prune_tau;
+  int32_t skip_cap;
 } ks_params;
 
 /* Outputs of ks_solve: caller-allocated DEVICE buffers.  C = K + 1 cells,

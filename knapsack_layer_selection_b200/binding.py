@@ -49,7 +49,8 @@ class Params(ctypes.Structure):
     _fields_ = [("gamma_max", ctypes.c_int32), ("n_bins", ctypes.c_int32),
                 ("budget_mode", ctypes.c_int32),
                 ("alpha_lo", ctypes.c_double), ("alpha_scale", ctypes.c_double),
-                ("alpha_max", ctypes.c_double)]
+                ("alpha_max", ctypes.c_double), ("prune_tau", ctypes.c_double),
+                ("skip_cap", ctypes.c_int32)]
 
 
 class Result(ctypes.Structure):
@@ -163,9 +164,12 @@ def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int) -> CacheD
 
 
 def params(gamma_max: int, n_bins: int = 0, alpha_lo: float = 0.5, alpha_scale: float = 0.5,
-           alpha_max: float = 0.99, budget_mode: str = "at_most") -> Params:
+           alpha_max: float = 0.99, budget_mode: str = "at_most",
+           prune_tau: Optional[float] = None, skip_cap: Optional[int] = None) -> Params:
     mode = {"at_most": KS_BUDGET_AT_MOST, "exact": KS_BUDGET_EXACT}[budget_mode]
-    return Params(gamma_max, n_bins, mode, alpha_lo, alpha_scale, alpha_max)
+    return Params(gamma_max, n_bins, mode, alpha_lo, alpha_scale, alpha_max,
+                  float("-inf") if prune_tau is None else float(prune_tau),
+                  -1 if skip_cap is None else int(skip_cap))
 
 
 # ---------------------------------------------------------------- calls

@@ -460,6 +460,8 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     return fail(KS_ERR_INVALID_ARG, "solve: gamma_max >= 1 and alpha_scale > 0");
   if (params->budget_mode != KS_BUDGET_AT_MOST && params->budget_mode != KS_BUDGET_EXACT)
     return fail(KS_ERR_INVALID_ARG, "solve: budget_mode must be KS_BUDGET_AT_MOST or KS_BUDGET_EXACT");
+  if (params->prune_tau != params->prune_tau)
+    return fail(KS_ERR_INVALID_ARG, "solve: prune_tau is NaN (use -INFINITY to turn it off)");
   const int n_items = 2 * model->n_layers;
   std::vector<int32_t> ww;
   KS_TRY(resolve_weights(n_items, w, t, params, &ww));
@@ -500,12 +502,18 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   float* cur = c.ws.cur;
   uint8_t* bp = out->bp ? out->bp : c.ws.bp;
   const bool exact = params->budget_mode == KS_BUDGET_EXACT;
-  uint8_t* vprev = exact ? c.ws.valid_a : nullptr;
-  uint8_t* vcur = exact ? c.ws.valid_b : nullptr;
-  if (exact) KS_TRY(launch_init_valid(vprev, C, st));
+  const bool pruning = params->prune_tau > -INFINITY || params->skip_cap >= 0;
+  const bool track = exact || pruning;       // validity is carried only when it can change
+  uint8_t* vprev = track ? c.ws.valid_a : nullptr;
+  uint8_t* vcur = track ? c.ws.valid_b : nullptr;
+  if (track) KS_TRY(launch_init_valid(vprev, C, exact, st));
+  long long W_k = 0;                          // cumulative weight through item k
   for (int k = 0; k < n_items; ++k) {
     const int wk = ww[k];
     const int E = C - wk;
+    W_k += wk;
+    const int min_valid_b =
+        params->skip_cap >= 0 ? (int)std::max(0LL, W_k - (long long)params->skip_cap) : 0;
     KS_TRY(sublayer(c, k, prev, E + 1, c.ws.exec, /*xh_ready=*/true));
     float* val = (k == n_items - 1) ? out->values : c.ws.val;
     const void* g_next = nullptr;
@@ -519,7 +527,7 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
                                out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
                                out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
                                out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr,
-                               vprev, vcur, st));
+                               vprev, vcur, params->prune_tau, min_valid_b, st));
     std::swap(prev, cur);
     std::swap(vprev, vcur);
   }

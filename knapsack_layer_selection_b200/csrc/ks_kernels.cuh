@@ -55,7 +55,8 @@ ks_status launch_select_fused(const float* prev, const float* exec, const float*
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
-                              uint8_t* valid_cur, cudaStream_t st);
+                              uint8_t* valid_cur, double prune_tau, int min_valid_b,
+                              cudaStream_t st);
 
 // Slots 0..n_slots-1 of a state buffer <- x0, and their normalised operands.
 ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
@@ -73,8 +74,8 @@ ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* 
                              int32_t* used_w, double* t_draft, int32_t* status,
                              const uint8_t* valid, cudaStream_t st);
 
-// valid[b] = (b == 0) for the exact-budget mode.
-ks_status launch_init_valid(uint8_t* valid, int C, cudaStream_t st);
+// Initial validity: only b == 0 in the exact-budget mode, every cell otherwise.
+ks_status launch_init_valid(uint8_t* valid, int C, bool exact, cudaStream_t st);
 
 ks_status launch_tpt(const float* values, const double* t_draft, int C, double t_target,
                      int gamma_max, double lo, double scale, double amax, double* tpt,

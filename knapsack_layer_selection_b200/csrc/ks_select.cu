@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
     const TG* __restrict__ g_next, float* __restrict__ cur, TX* __restrict__ xh_next,
     float* __restrict__ val, uint8_t* __restrict__ bp, float* __restrict__ cos_s_out,
     float* __restrict__ cos_e_out, float* __restrict__ ref_out,
-    const uint8_t* __restrict__ valid_prev, uint8_t* __restrict__ valid_cur) {
+    const uint8_t* __restrict__ valid_prev, uint8_t* __restrict__ valid_cur, double prune_tau,
+    int min_valid_b) {
   __shared__ double cs_tok[kSelectMaxT];
   __shared__ double ce_tok[kSelectMaxT];
   __shared__ float inv_s[kSelectMaxT];
@@ -202,10 +203,13 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
       const bool sv = valid_prev ? valid_prev[b] != 0 : true;
       const bool ev = has_e && (valid_prev ? valid_prev[b - w] != 0 : true);
       take = ev && (!sv || me > ms) ? 1 : 0;
+      const double kept = take ? me : ms;
+      // pruning: a kept value below tau, or a budget below W_k - cap, drops the cell
+      const bool alive = (sv || ev) && !(kept < prune_tau) && b >= min_valid_b;
       const float nan = __int_as_float(0x7fc00000);
-      val[b] = (sv || ev) ? (float)(take ? me : ms) : nan;
+      val[b] = alive ? (float)kept : nan;
       bp[b] = (uint8_t)take;
-      if (valid_cur) valid_cur[b] = (uint8_t)(sv || ev);
+      if (valid_cur) valid_cur[b] = (uint8_t)alive;
       if (cos_s_out) cos_s_out[b] = sv ? (float)ms : nan;
       if (cos_e_out) cos_e_out[b] = ev ? (float)me : nan;
     }
@@ -236,17 +240,19 @@ ks_status launch_select_fused(const float* prev, const float* exec, const float*
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
-                              uint8_t* valid_cur, cudaStream_t st) {
+                              uint8_t* valid_cur, double prune_tau, int min_valid_b,
+                              cudaStream_t st) {
   if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "select: T above 256");
   if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "select: d must be a multiple of 4");
   if (wdt == KS_BF16)
     select_fused_kernel<__nv_bfloat16, __nv_bfloat16><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const __nv_bfloat16*)g_next, cur,
-        (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out, valid_prev, valid_cur);
+        (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out, valid_prev, valid_cur,
+        prune_tau, min_valid_b);
   else
     select_fused_kernel<float, float><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const float*)g_next, cur, (float*)xh_next, val, bp,
-        cos_s, cos_e, ref_out, valid_prev, valid_cur);
+        cos_s, cos_e, ref_out, valid_prev, valid_cur, prune_tau, min_valid_b);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -357,13 +363,13 @@ ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* 
   return KS_OK;
 }
 
-__global__ void init_valid_kernel(uint8_t* valid, int C) {
+__global__ void init_valid_kernel(uint8_t* valid, int C, int exact) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < C) valid[b] = (uint8_t)(b == 0);
+  if (b < C) valid[b] = (uint8_t)(exact ? b == 0 : 1);
 }
 
-ks_status launch_init_valid(uint8_t* valid, int C, cudaStream_t st) {
-  init_valid_kernel<<<ceil_div(C, 256), 256, 0, st>>>(valid, C);
+ks_status launch_init_valid(uint8_t* valid, int C, bool exact, cudaStream_t st) {
+  init_valid_kernel<<<ceil_div(C, 256), 256, 0, st>>>(valid, C, exact ? 1 : 0);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }

@@ -46,6 +46,8 @@ R12 alpha_S = clamp((value - lo) / scale, 0, alpha_max) (a stated stand-in for
    the paper's history-based estimate, Eq. 9).
 R13 TPT ties: larger TPT, then smaller b, then smaller gamma.
 R14 b = 0 (the empty set) takes part in the grid search.
+R15 cosine pruning (optional): a cell whose kept value is below tau is dropped.
+R16 skip cap (optional): after item k the cells b < W_k - cap are dropped.
 
 Item numbering: items k = 0 .. 2L-1; item 2l is the Attention sublayer of
 layer l and item 2l+1 its MLP sublayer.  X^(0) is the evaluation tokens' input
@@ -255,7 +257,9 @@ class DPResult:
 def knapsack_dp(w: Sequence[int], n_cells: int, init_states: np.ndarray,
                 init_valid: np.ndarray,
                 item_fn: Callable[[int, np.ndarray], np.ndarray],
-                score_fn: Callable[[int, np.ndarray], np.ndarray]) -> DPResult:
+                score_fn: Callable[[int, np.ndarray], np.ndarray],
+                prune: Optional[Callable[[int, np.ndarray, np.ndarray], np.ndarray]] = None
+                ) -> DPResult:
     """Row-by-row 0/1-knapsack DP that keeps one state per (item, budget) cell.
 
     Eq. 7/8 and Algorithm 1 as the review describes them (referee major 1 and
@@ -264,7 +268,10 @@ def knapsack_dp(w: Sequence[int], n_cells: int, init_states: np.ndarray,
     applied to the previous row's state at b - w_k (reading R2); the candidate
     with the larger score is kept, execute only when strictly larger (R3), and
     the choice is stored as a backpointer (R4).  ``score_fn(k+1, states)``
-    scores states against the target of row k+1.
+    scores states against the target of row k+1.  ``prune(k+1, values,
+    valid)`` may then drop cells of the new row (they become invalid: no
+    later candidate reads them); it is how the review's cosine threshold and
+    skipped-weight cap (R15, R16) enter.
     """
     n_items = len(w)
     C = n_cells
@@ -299,6 +306,9 @@ def knapsack_dp(w: Sequence[int], n_cells: int, init_states: np.ndarray,
                         cur_valid[b] = True
                         cur_val[b] = e
                         bp[k, b] = 1
+        if prune is not None:
+            cur_valid = np.asarray(prune(k + 1, cur_val, cur_valid), dtype=bool)
+            cur_val = np.where(cur_valid, cur_val, np.nan)
         prev, valid = cur, cur_valid
         val[k + 1] = cur_val
         vrows[k + 1] = valid
@@ -345,12 +355,21 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
              gamma_max: int, n_cells: Optional[int] = None, mode: str = "at_most",
              per_cell: bool = False, ref: Optional[np.ndarray] = None,
              alpha_lo: float = 0.5, alpha_scale: float = 0.5, alpha_max: float = 0.99,
-             keep_states: bool = False) -> Solve:
+             keep_states: bool = False, prune_tau: Optional[float] = None,
+             skip_cap: Optional[int] = None) -> Solve:
     """KnapSpec's DP over all budget cells, reconstruction and TPT selection.
 
     ``n_cells`` < K+1 computes only the budgets 0 .. n_cells-1, which equal the
     full DP's cells there (every read goes to an equal or smaller budget).  The
     TPT search then runs over those cells only.
+
+    ``prune_tau`` drops a cell whose kept value is below tau (the review's
+    cosine threshold tau = 0.5, "Assumptions & free parameters" and referee
+    notes on Fig. 4; reading R15); ``skip_cap`` drops, after item k, the cells
+    b < W_k - cap, W_k = w_0 + .. + w_k (the skipped-weight cap K/2 of the
+    review's "Reading between the lines"; reading R16).  A dropped cell is
+    invalid: its value is NaN, no later candidate reads it, and a final
+    invalid cell has no set.
     """
     x0 = np.asarray(x0, F64)
     n_items = model.n_items
@@ -372,7 +391,8 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
 
     dp = knapsack_dp(w, C, init, init_valid,
                      lambda k, H: apply_item(model, k, H, ctx, per_cell=per_cell),
-                     lambda r, H: meancos(H, ref[r]))
+                     lambda r, H: meancos(H, ref[r]),
+                     prune=pruning_rule(w, C, prune_tau, skip_cap))
     sets, used = [], np.zeros(C, dtype=np.int64)
     t_draft = np.zeros(C)
     for b in range(C):
@@ -399,6 +419,30 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
     out.tpt = grid
     out.best_b, out.best_gamma, out.best_tpt = tpt_argmax(grid)
     return out
+
+
+def pruning_rule(w: Sequence[int], n_cells: int, prune_tau: Optional[float],
+                 skip_cap: Optional[int]):
+    """The prune callback of knapsack_dp for a cosine threshold and a skip cap.
+
+    After item k (row r = k + 1): a cell stays valid only if its value is not
+    below tau and its budget b is at least W_k - cap (a cell below that bound
+    has skipped more than cap weight units whatever its exact usage).
+    """
+    if prune_tau is None and skip_cap is None:
+        return None
+    W = np.cumsum(np.asarray(w, dtype=np.int64))
+    cells = np.arange(n_cells)
+
+    def prune(r, vals, valid):
+        v = np.array(valid, dtype=bool, copy=True)
+        if skip_cap is not None:
+            v &= cells >= W[r - 1] - int(skip_cap)
+        if prune_tau is not None:
+            v &= ~(np.nan_to_num(vals, nan=np.inf) < float(prune_tau))
+        return v
+
+    return prune
 
 
 # --------------------------------------------------------------------------
@@ -508,7 +552,8 @@ def brute_force(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], ref: n
 # Scalar special case: the DP skeleton on numbers is the textbook 0/1 knapsack
 # --------------------------------------------------------------------------
 def scalar_knapsack_dp(w: Sequence[int], v: Sequence[int], capacity: int,
-                       mode: str = "at_most") -> Tuple[np.ndarray, DPResult]:
+                       mode: str = "at_most", prune_tau: Optional[float] = None,
+                       skip_cap: Optional[int] = None) -> Tuple[np.ndarray, DPResult]:
     """The same DP skeleton with state = running value, item(k, x) = x + v_k, score = x.
 
     With additive item values the keep-the-better rule is exactly the classic
@@ -524,6 +569,7 @@ def scalar_knapsack_dp(w: Sequence[int], v: Sequence[int], capacity: int,
         iv = np.zeros(C, dtype=bool)
         iv[0] = True
     vv = np.asarray(v, F64)
-    res = knapsack_dp(w, C, init, iv, lambda k, H: H + vv[k], lambda r, H: np.asarray(H, F64))
+    res = knapsack_dp(w, C, init, iv, lambda k, H: H + vv[k], lambda r, H: np.asarray(H, F64),
+                      prune=pruning_rule(w, C, prune_tau, skip_cap))
     vals = np.where(res.valid[len(w)], res.val[len(w)], -np.inf)
     return vals, res

@@ -40,13 +40,17 @@ class Report:
         assert self.argmax_ok, self
 
 
-def taint_mask(w, bp_o, bp_g, cos_s_o, cos_e_o):
+def taint_mask(w, bp_o, bp_g, cos_s_o, cos_e_o, extra=None):
+    """extra [n][C]: cells tainted whatever their backpointers (e.g. values within
+    the near-tie distance of a pruning threshold, whose validity may flip)."""
     n, C = bp_o.shape
     near = np.abs(np.nan_to_num(cos_e_o, nan=np.inf) - np.nan_to_num(cos_s_o, nan=-np.inf)) < NEAR_TIE
     taint = np.zeros((n, C), dtype=bool)
     prev = np.zeros(C, dtype=bool)
     for k in range(n):
         t = near[k] & (bp_o[k] != bp_g[k])
+        if extra is not None:
+            t |= extra[k]
         t |= prev
         wk = int(w[k])
         if wk < C:
@@ -57,14 +61,18 @@ def taint_mask(w, bp_o, bp_g, cos_s_o, cos_e_o):
 
 
 def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=None,
-                  check_argmax=True) -> Report:
+                  check_argmax=True, prune_tau=None) -> Report:
     """orc: oracle Solve; gpu: dict of numpy arrays bp [n][C], values [C], sets (lists),
     best (b, gamma), tpt grid [C][G] (optional); rows_val_gpu: [n][C] chosen values.
     With check_argmax=False (a budget prefix) the TPT choice is not compared."""
     bp_o = orc.dp.bp
     C = bp_o.shape[1]
     bp_g = gpu["bp"]
-    near, taint = taint_mask(w, bp_o, bp_g, orc.dp.cos_s, orc.dp.cos_e)
+    extra = None
+    if prune_tau is not None:
+        kept = np.where(bp_o == 1, orc.dp.cos_e, orc.dp.cos_s)
+        extra = np.abs(np.nan_to_num(kept, nan=np.inf) - prune_tau) < NEAR_TIE
+    near, taint = taint_mask(w, bp_o, bp_g, orc.dp.cos_s, orc.dp.cos_e, extra)
     r = Report(n_cells=C)
     r.near_ties = int(near.sum())
     r.tainted = int(taint.sum())
@@ -85,7 +93,7 @@ def compare_solve(orc, gpu, w, val_tol, n_items, sets_gpu=None, rows_val_gpu=Non
     r.val_fail = int(np.sum(err[ok] > val_tol))
     if rows_val_gpu is not None:
         e2 = errors(rows_val_gpu, orc.dp.val[1:])
-        m = ~taint
+        m = ~taint & orc.dp.valid[1:]
         r.val_max_err = max(r.val_max_err, float(np.max(e2[m])) if m.any() else 0.0)
         r.val_fail += int(np.sum(e2[m] > val_tol))
     sets_g = gpu["sets"]

@@ -28,11 +28,11 @@ def lib():
     return B.load()
 
 
-def make_solver(wl, inp_gpu, w=None, t=None, keep_cos=True, mode="at_most"):
+def make_solver(wl, inp_gpu, w=None, t=None, keep_cos=True, mode="at_most", tau=None, cap=None):
     m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
                      wl.rms_eps, wl.rope_base, wl.wdtype)
     t = wl.latencies() if t is None else t
-    prm = B.params(wl.gamma_max, wl.n_bins, budget_mode=mode)
+    prm = B.params(wl.gamma_max, wl.n_bins, budget_mode=mode, prune_tau=tau, skip_cap=cap)
     return B.Solver(m, inp_gpu.layers, inp_gpu.k_cache, inp_gpu.v_cache, wl.ctx, wl.T, t, prm,
                     w=w, keep_cos=keep_cos)
 
@@ -53,8 +53,8 @@ def gpu_result(solver):
 _cache = {}
 
 
-def solved(name, n_layers=None, mode="at_most"):
-    key = (name, n_layers, mode)
+def solved(name, n_layers=None, mode="at_most", tau=None, cap=None):
+    key = (name, n_layers, mode, tau, cap)
     if key in _cache:
         return _cache[key]
     wl = W.WORKLOADS[name]
@@ -66,11 +66,11 @@ def solved(name, n_layers=None, mode="at_most"):
         wl = inp.wl
         t, w = t[:2 * n_layers], w[:2 * n_layers]
     g = inp.to("cuda")
-    solver = make_solver(wl, g, w=w, t=t, mode=mode)
+    solver = make_solver(wl, g, w=w, t=t, mode=mode, tau=tau, cap=cap)
     solver.solve(g.x0)
     res = gpu_result(solver)
     orc = O.dp_solve(oracle_model(inp), x0_np(inp), wl.ctx, w, t, wl.gamma_max,
-                     per_cell=(wl.wdtype == "f32"), mode=mode)
+                     per_cell=(wl.wdtype == "f32"), mode=mode, prune_tau=tau, skip_cap=cap)
     _cache[key] = (wl, inp, g, solver, res, orc, w, t)
     return _cache[key]
 
@@ -110,6 +110,35 @@ def test_exact_budget_mode_matches_oracle(name, n_layers):
             assert res["used_w"][b] == -1 and res["sets"][b] == []
     # reachable budgets are exactly the subset sums
     assert abs(res["values"][-1] - 1.0) <= 1e-6
+
+
+PRUNE_CASES = [("tiny", None, "at_most", 0.9992, None), ("tiny", None, "exact", None, 14),
+               ("small", 4, "at_most", 0.8, 32), ("small", None, "at_most", 0.85, 128),
+               ("small", None, "exact", 0.85, 128)]
+
+
+@pytest.mark.parametrize("name,n_layers,mode,tau,cap", PRUNE_CASES)
+def test_pruning_rules_match_oracle(name, n_layers, mode, tau, cap):
+    """Cosine threshold and skip cap (the review's tau and K/2): the cells each
+    rule drops must be the oracle's, up to cells whose value is within the
+    near-tie distance of tau (treated like near-ties)."""
+    wl, inp, g, solver, res, orc, w, t = solved(name, n_layers, mode, tau, cap)
+    rep = compare_solve(orc, res, w, VAL_TOL[wl.wdtype], wl.n_items, rows_val_gpu=res["rows"],
+                        prune_tau=tau)
+    valid_o = orc.dp.valid[-1]
+    dropped = int((~valid_o).sum())
+    print(f"\n{name}/{n_layers} {mode} tau={tau} cap={cap}: {dropped} of {len(valid_o)} final "
+          f"cells dropped; {rep}")
+    rep.assert_ok()
+    ok = ~np.isnan(orc.values) | ~np.isnan(res["values"])
+    kept = np.where(orc.dp.bp == 1, orc.dp.cos_e, orc.dp.cos_s)
+    near = (np.abs(np.nan_to_num(kept, nan=np.inf) - (tau if tau is not None else -9)) < 1e-4).any(0)
+    # validity agrees wherever no near-threshold cell could have flipped it
+    if not near.any():
+        assert np.array_equal(np.isnan(res["values"]), np.isnan(orc.values))
+    if cap is not None:
+        K = sum(w)
+        assert np.all(np.isnan(res["values"][:max(0, K - cap)]))
 
 
 def test_small_first_8_items_bounded_by_exhaustive_search():

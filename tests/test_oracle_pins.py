@@ -394,11 +394,88 @@ def test_planted_dp_index_error_is_caught(monkeypatch):
     """Executing from cell b - w + 1 instead of b - w breaks the knapsack optimum."""
     good = O.knapsack_dp
 
-    def bad(w, n_cells, init_states, init_valid, item_fn, score_fn):
-        return good([max(1, x - 1) for x in w], n_cells, init_states, init_valid, item_fn, score_fn)
+    def bad(w, n_cells, init_states, init_valid, item_fn, score_fn, prune=None):
+        return good([max(1, x - 1) for x in w], n_cells, init_states, init_valid, item_fn,
+                    score_fn, prune)
 
     monkeypatch.setattr(O, "knapsack_dp", bad)
     g = json.load(open(os.path.join(GOLDEN, "knapsack_textbook.json")))
     cap = len(g["at_most_best"]) - 1
     vals, _ = O.scalar_knapsack_dp(g["weights"], g["values"], cap, "at_most")
     assert vals.tolist() != [float(x) for x in g["at_most_best"]]
+
+
+# ---------------------------------------------------------------- pruning rules (R15, R16)
+def _recursive_pruned_dp(w, v, cap_b, mode, tau, skip_cap):
+    """The same rule written top-down with memoisation: V(i, b) -> (valid, value)."""
+    import functools
+    W = np.cumsum(w)
+
+    @functools.lru_cache(maxsize=None)
+    def V(i, b):
+        if i == 0:
+            return (mode == "at_most" or b == 0, 0.0)
+        sv, s_val = V(i - 1, b)
+        ev, e_val = (False, 0.0)
+        if b >= w[i - 1]:
+            src_v, src = V(i - 1, b - w[i - 1])
+            ev, e_val = src_v, src + v[i - 1]
+        if ev and (not sv or e_val > s_val):
+            ok, val = True, e_val
+        elif sv:
+            ok, val = True, s_val
+        else:
+            return (False, 0.0)
+        if skip_cap is not None and b < W[i - 1] - skip_cap:
+            ok = False
+        if tau is not None and val < tau:
+            ok = False
+        return (ok, val)
+
+    out = []
+    for b in range(cap_b + 1):
+        ok, val = V(len(w), b)
+        out.append(val if ok else -math.inf)
+    return out
+
+
+@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("mode", ["at_most", "exact"])
+def test_pruning_rules_match_recursive_definition(seed, mode):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(2, 10))
+    w = rng.integers(1, 6, size=n).tolist()
+    v = rng.integers(-4, 9, size=n).tolist()
+    cap = int(sum(w))
+    tau = float(rng.integers(-3, 6))
+    skip = int(rng.integers(0, cap + 1))
+    for t_, s_ in [(tau, None), (None, skip), (tau, skip)]:
+        vals, _ = O.scalar_knapsack_dp(w, v, cap, mode, prune_tau=t_, skip_cap=s_)
+        assert vals.tolist() == _recursive_pruned_dp(w, v, cap, mode, t_, s_), (t_, s_)
+
+
+def test_skip_cap_in_exact_mode_only_removes_unreachable_budgets(tiny):
+    """Exact budgets: a final cell b is reachable within a cap c iff b >= K - c, and the
+    cap removes nothing else (skipped weight only grows along a path)."""
+    wl, inp, m = tiny
+    t = wl.latencies()
+    w = O.quantize_weights(t, wl.n_bins)
+    K = sum(w)
+    full = O.dp_solve(m, x0_np(inp), wl.ctx, w, t, wl.gamma_max, mode="exact")
+    cap = K // 2
+    capped = O.dp_solve(m, x0_np(inp), wl.ctx, w, t, wl.gamma_max, mode="exact", skip_cap=cap)
+    for b in range(K + 1):
+        if b >= K - cap:
+            assert np.array_equal(np.isnan(full.values[b]), np.isnan(capped.values[b]))
+            if np.isfinite(full.values[b]):
+                assert capped.values[b] == full.values[b] and capped.sets[b] == full.sets[b]
+        else:
+            assert np.isnan(capped.values[b])
+
+
+def test_disabled_rules_change_nothing(tiny, tiny_solve):
+    wl, inp, m = tiny
+    s = tiny_solve
+    p = O.dp_solve(m, x0_np(inp), wl.ctx, s.w, s.t, wl.gamma_max, per_cell=True,
+                   prune_tau=-np.inf, skip_cap=sum(s.w))
+    assert np.array_equal(p.dp.bp, s.dp.bp) and np.array_equal(p.values, s.values)
