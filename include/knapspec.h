@@ -134,6 +134,11 @@ typedef struct {
    * W_k = w_0 + .. + w_k.  prune_tau = -INFINITY and skip_cap < 0 turn them off. */
   double prune_tau;
   int32_t skip_cap;
+  /* Distinct-state execution: before each item, budget cells whose states are
+   * bit-for-bit equal (and valid) are folded together and the item runs once
+   * per distinct state.  Results are identical to the dense solve (every row's
+   * arithmetic is independent of its batch); only the work shrinks.  0 = off. */
+  int32_t dedup;
 } ks_params;
 
 /* Outputs of ks_solve: caller-allocated DEVICE buffers.  C = K + 1 cells,
@@ -152,6 +157,8 @@ typedef struct {
   double* best_tpt;    /* [1] optional: TPT(b*, gamma*) */
   float* ref_states;   /* [n_items+1][T][d] optional: the full model's states X^(k)
                           the solve computed (they ride along in each item's batch) */
+  int32_t* exec_counts; /* [n_items] optional: states item k ran on (with dedup: the
+                           distinct ones, the reference included) */
 } ks_result;
 
 /* Library version string (static storage). */

@@ -50,13 +50,13 @@ class Params(ctypes.Structure):
                 ("budget_mode", ctypes.c_int32),
                 ("alpha_lo", ctypes.c_double), ("alpha_scale", ctypes.c_double),
                 ("alpha_max", ctypes.c_double), ("prune_tau", ctypes.c_double),
-                ("skip_cap", ctypes.c_int32)]
+                ("skip_cap", ctypes.c_int32), ("dedup", ctypes.c_int32)]
 
 
 class Result(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("status", "values", "sets", "used_w", "t_draft", "bp", "cos_skip",
-                 "cos_exec", "tpt", "best", "best_tpt", "ref_states")]
+                 "cos_exec", "tpt", "best", "best_tpt", "ref_states", "exec_counts")]
 
 
 class KernelStat(ctypes.Structure):
@@ -165,11 +165,12 @@ def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int) -> CacheD
 
 def params(gamma_max: int, n_bins: int = 0, alpha_lo: float = 0.5, alpha_scale: float = 0.5,
            alpha_max: float = 0.99, budget_mode: str = "at_most",
-           prune_tau: Optional[float] = None, skip_cap: Optional[int] = None) -> Params:
+           prune_tau: Optional[float] = None, skip_cap: Optional[int] = None,
+           dedup: bool = False) -> Params:
     mode = {"at_most": KS_BUDGET_AT_MOST, "exact": KS_BUDGET_EXACT}[budget_mode]
     return Params(gamma_max, n_bins, mode, alpha_lo, alpha_scale, alpha_max,
                   float("-inf") if prune_tau is None else float(prune_tau),
-                  -1 if skip_cap is None else int(skip_cap))
+                  -1 if skip_cap is None else int(skip_cap), 1 if dedup else 0)
 
 
 # ---------------------------------------------------------------- calls
@@ -310,6 +311,7 @@ class SolveOutputs:
     cos_exec: Optional[torch.Tensor] = None
     tpt: Optional[torch.Tensor] = None
     ref_states: Optional[torch.Tensor] = None
+    exec_counts: Optional[torch.Tensor] = None
 
 
 class Solver:
@@ -346,12 +348,13 @@ class Solver:
             cos_skip=z(n, C, dt=torch.float32) if keep_cos else None,
             cos_exec=z(n, C, dt=torch.float32) if keep_cos else None,
             tpt=z(C, prm.gamma_max, dt=torch.float64) if keep_tpt else None,
-            ref_states=z(n + 1, T, model.d_model, dt=torch.float32) if keep_ref else None)
+            ref_states=z(n + 1, T, model.d_model, dt=torch.float32) if keep_ref else None,
+            exec_counts=z(n, dt=torch.int32))
         o = self.out
         p = lambda x: None if x is None else x.data_ptr()
         self.result = Result(p(o.status), p(o.values), p(o.sets), p(o.used_w), p(o.t_draft),
                              p(o.bp), p(o.cos_skip), p(o.cos_exec), p(o.tpt), p(o.best),
-                             p(o.best_tpt), p(o.ref_states))
+                             p(o.best_tpt), p(o.ref_states), p(o.exec_counts))
         self._t_arr = (ctypes.c_double * n)(*self.t)
         self._w_arr = (ctypes.c_int32 * n)(*self.w)
 

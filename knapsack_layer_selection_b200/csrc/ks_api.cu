@@ -80,6 +80,10 @@ struct Workspace {
   void *gb, *ub;              // [(C+1)T][ffn] act
   uint8_t* bp;                // [n_items][C]
   uint8_t *valid_a, *valid_b; // [C] exact-budget validity, ping-pong
+  uint64_t *hash_a, *hash_b;  // [C+1] state fingerprints (distinct-state execution), ping-pong
+  int *map, *uniq, *count;    // [C+1], [C+1], [1] compaction of the execute batch
+  float* prev_c;              // [C+1][T][d] fp32 distinct source states
+  void* xh_c;                 // [C+1][T][d] act: their normalised operands
   float* val;                 // [C]
   double* t_draft;            // [C]
   float2* rope;               // [T][hd/2]
@@ -115,6 +119,13 @@ static Workspace carve(const ks_model_desc* m, long long n_slots, long long T, c
   w.bp = (uint8_t*)take(n_items * C);
   w.valid_a = (uint8_t*)take(C);
   w.valid_b = (uint8_t*)take(C);
+  w.hash_a = (uint64_t*)take((C + 1) * 8);
+  w.hash_b = (uint64_t*)take((C + 1) * 8);
+  w.map = (int*)take((C + 1) * 4);
+  w.uniq = (int*)take((C + 1) * 4);
+  w.count = (int*)take(4);
+  w.prev_c = (float*)take(R * d * 4);
+  w.xh_c = take(R * d * ab);
   w.val = (float*)take(C * 4);
   w.t_draft = (double*)take(C * 8);
   w.rope = (float2*)take(T * (m->head_dim / 2) * sizeof(float2));
@@ -138,7 +149,8 @@ struct Ctx {
 // The RoPE table in ws.rope must hold positions ctx .. ctx+T-1.  With
 // xh_ready, ws.xh already holds the item's normalised operand of `in`.
 static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* out,
-                          bool xh_ready = false) {
+                          bool xh_ready = false, const void* xh_src = nullptr,
+                          const int* dyn_cells = nullptr) {
   const ks_model_desc* m = c.m;
   const int l = k / 2;
   const ks_layer_weights& L = c.layers[l];
@@ -149,6 +161,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
   const double ab = (double)act_bytes(c.act);
   const double wb = m->wdtype == KS_F32 ? 4.0 : 2.0;
   const double Rd = (double)R;
+  const void* xh = xh_src ? xh_src : c.ws.xh;   // the item's normalised operand
   if (!xh_ready) {
     ProfScope ps(KK_RMSNORM, c.st, 3.0 * Rd * d, Rd * d * (4.0 + ab));
     KS_TRY(launch_rmsnorm(in, k % 2 == 0 ? L.attn_norm : L.mlp_norm, m->wdtype, c.ws.xh, c.act, R,
@@ -164,10 +177,10 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
       ProfScope ps(KK_GEMM_Q, c.st, 2.0 * Rd * qd * d, (Rd * d + (double)qd * d) * ab + Rd * qd * ab,
                    tc ? 1 : 2);
       if (tc) {
-        KS_TRY(tc_gemm(c.ws.xh, L.wq, nullptr, c.ws.q, nullptr, R, qd, d, EPI_ROPE_BF16, c.ws.rope,
-                       c.T, m->head_dim, c.status, c.st));
+        KS_TRY(tc_gemm(xh, L.wq, nullptr, c.ws.q, nullptr, R, qd, d, EPI_ROPE_BF16, c.ws.rope,
+                       c.T, m->head_dim, c.status, c.st, dyn_cells));
       } else {
-        KS_TRY(launch_gemm_simt(c.ws.xh, c.act, L.wq, m->wdtype, c.ws.q, false, nullptr, R, qd, d,
+        KS_TRY(launch_gemm_simt(xh, c.act, L.wq, m->wdtype, c.ws.q, false, nullptr, R, qd, d,
                                 c.st));
         KS_TRY(launch_rope_inplace(c.ws.q, c.act, c.ws.rope, R, m->n_q_heads, m->head_dim, c.T,
                                    c.st));
@@ -181,7 +194,8 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                    2.0 * Rd * qd * ab + kv_bytes);
       if (tc) {
         KS_TRY(tc_attention(c.ws.q, kc, vc, c.cache->cache_rows, R, c.T, m->n_q_heads,
-                            m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.status, c.st));
+                            m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.status, c.st,
+                            dyn_cells));
       } else {
         KS_TRY(launch_attention_simt(c.ws.q, c.act, kc, vc, m->wdtype, R, c.T, m->n_q_heads,
                                      m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.st));
@@ -192,7 +206,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                    (Rd * qd + (double)d * qd) * ab + Rd * d * 8.0);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.att, L.wo, nullptr, out, in, R, d, qd, EPI_RESID_F32, nullptr, c.T,
-                       m->head_dim, c.status, c.st));
+                       m->head_dim, c.status, c.st, dyn_cells));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.att, c.act, L.wo, m->wdtype, out, true, in, R, d, qd, c.st));
       }
@@ -203,12 +217,12 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
       ProfScope ps(KK_GEMM_GATEUP, c.st, 2.0 * Rd * 2.0 * F * d,
                    (Rd * d + 2.0 * F * d) * ab + Rd * F * ab, tc ? 1 : 3);
       if (tc) {
-        KS_TRY(tc_gemm(c.ws.xh, L.w_gate, L.w_up, c.ws.gb, nullptr, R, F, d, EPI_SWIGLU_BF16,
-                       nullptr, c.T, m->head_dim, c.status, c.st));
+        KS_TRY(tc_gemm(xh, L.w_gate, L.w_up, c.ws.gb, nullptr, R, F, d, EPI_SWIGLU_BF16,
+                       nullptr, c.T, m->head_dim, c.status, c.st, dyn_cells));
       } else {
-        KS_TRY(launch_gemm_simt(c.ws.xh, c.act, L.w_gate, m->wdtype, c.ws.gb, false, nullptr, R, F,
+        KS_TRY(launch_gemm_simt(xh, c.act, L.w_gate, m->wdtype, c.ws.gb, false, nullptr, R, F,
                                 d, c.st));
-        KS_TRY(launch_gemm_simt(c.ws.xh, c.act, L.w_up, m->wdtype, c.ws.ub, false, nullptr, R, F,
+        KS_TRY(launch_gemm_simt(xh, c.act, L.w_up, m->wdtype, c.ws.ub, false, nullptr, R, F,
                                 d, c.st));
         KS_TRY(launch_swiglu_inplace(c.ws.gb, c.ws.ub, c.act, (long long)R * F, c.st));
       }
@@ -217,7 +231,7 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
       ProfScope ps(KK_GEMM_DOWN, c.st, 2.0 * Rd * d * F, (Rd * F + (double)d * F) * ab + Rd * d * 8.0);
       if (tc) {
         KS_TRY(tc_gemm(c.ws.gb, L.w_down, nullptr, out, in, R, d, F, EPI_RESID_F32, nullptr, c.T,
-                       m->head_dim, c.status, c.st));
+                       m->head_dim, c.status, c.st, dyn_cells));
       } else {
         KS_TRY(launch_gemm_simt(c.ws.gb, c.act, L.w_down, m->wdtype, out, true, in, R, d, F, c.st));
       }
@@ -493,10 +507,15 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   // the same batched kernels as the cells, so the select target X^(k+1) comes
   // out of each item's batch (exec slot 0) and no separate reference chain
   // runs.  Cells start from X^(0).
+  const bool dedup = params->dedup != 0;
+  if (dedup && C + 1 > 3072)
+    return fail(KS_ERR_UNSUPPORTED, "solve: distinct-state execution handles up to 3071 cells");
+  uint64_t* hprev = dedup ? c.ws.hash_a : nullptr;
+  uint64_t* hcur = dedup ? c.ws.hash_b : nullptr;
   {
     ProfScope ps(KK_BROADCAST, st, 0.0, (double)(C + 1) * cell * (4.0 + xb));
     KS_TRY(launch_init_states(x0, C + 1, T, model->d_model, model->rms_eps, layers[0].attn_norm,
-                              model->wdtype, c.ws.prev, c.ws.xh, out->ref_states, st));
+                              model->wdtype, c.ws.prev, c.ws.xh, out->ref_states, hprev, st));
   }
   float* prev = c.ws.prev;
   float* cur = c.ws.cur;
@@ -514,7 +533,24 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     W_k += wk;
     const int min_valid_b =
         params->skip_cap >= 0 ? (int)std::max(0LL, W_k - (long long)params->skip_cap) : 0;
-    KS_TRY(sublayer(c, k, prev, E + 1, c.ws.exec, /*xh_ready=*/true));
+    if (dedup) {
+      // fold equal source states together, then run the item once per distinct state
+      {
+        ProfScope ps(KK_DEDUP, st, 0.0, (E + 1.0) * 9.0);
+        KS_TRY(launch_dedup(hprev, vprev, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
+                            out->exec_counts ? out->exec_counts + k : nullptr, st));
+      }
+      {
+        ProfScope ps(KK_GATHER, st, 0.0, 2.0 * (E + 1.0) * cell * (4.0 + xb));
+        KS_TRY(launch_gather(c.ws.uniq, c.ws.count, E + 1, cell, prev, c.ws.xh, c.act, c.ws.prev_c,
+                             c.ws.xh_c, st));
+      }
+      KS_TRY(sublayer(c, k, c.ws.prev_c, E + 1, c.ws.exec, /*xh_ready=*/true, c.ws.xh_c,
+                      c.ws.count));
+    } else {
+      if (out->exec_counts) KS_TRY(launch_fill_i32(out->exec_counts + k, E + 1, st));
+      KS_TRY(sublayer(c, k, prev, E + 1, c.ws.exec, /*xh_ready=*/true));
+    }
     float* val = (k == n_items - 1) ? out->values : c.ws.val;
     const void* g_next = nullptr;
     if (k + 1 < n_items) g_next = (k + 1) % 2 == 0 ? layers[(k + 1) / 2].attn_norm
@@ -527,9 +563,11 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
                                out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
                                out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
                                out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr,
-                               vprev, vcur, params->prune_tau, min_valid_b, st));
+                               vprev, vcur, params->prune_tau, min_valid_b,
+                               dedup ? c.ws.map : nullptr, hcur, st));
     std::swap(prev, cur);
     std::swap(vprev, vcur);
+    std::swap(hprev, hcur);
   }
   double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;
   {

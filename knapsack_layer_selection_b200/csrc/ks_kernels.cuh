@@ -56,11 +56,19 @@ ks_status launch_select_fused(const float* prev, const float* exec, const float*
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
                               uint8_t* valid_cur, double prune_tau, int min_valid_b,
-                              cudaStream_t st);
+                              const int* exec_map, uint64_t* hash_cur, cudaStream_t st);
 
 // Slots 0..n_slots-1 of a state buffer <- x0, and their normalised operands.
 ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
-                             int wdt, float* states, void* xh, float* ref_out, cudaStream_t st);
+                             int wdt, float* states, void* xh, float* ref_out, uint64_t* hash_out,
+                             cudaStream_t st);
+
+// Distinct-state compaction of the next execute batch (slots 0..n-1): see ks_select.cu.
+ks_status launch_dedup(const uint64_t* hash, const uint8_t* valid, int n, int* map, int* uniq,
+                       int* count, int32_t* count_out, cudaStream_t st);
+ks_status launch_gather(const int* uniq, const int* count, int max_count, long long cell,
+                        const float* states, const void* xh, int act, float* states_c, void* xh_c,
+                        cudaStream_t st);
 
 struct ItemTable {
   static constexpr int kMaxItems = 256;
@@ -73,6 +81,9 @@ ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* 
                              const ItemTable* tab, int n_items, int C, uint64_t* sets,
                              int32_t* used_w, double* t_draft, int32_t* status,
                              const uint8_t* valid, cudaStream_t st);
+
+// *p = v (device word).
+ks_status launch_fill_i32(int32_t* p, int32_t v, cudaStream_t st);
 
 // Initial validity: only b == 0 in the exact-budget mode, every cell otherwise.
 ks_status launch_init_valid(uint8_t* valid, int C, bool exact, cudaStream_t st);

@@ -48,7 +48,8 @@ const char* kernel_kind_name(int k) {
   static const char* names[KK_COUNT] = {"rmsnorm", "gemm_q_rope", "gemm_o_residual",
                                         "gemm_gateup_swiglu", "gemm_down_residual", "rope",
                                         "swiglu", "attention", "select_bp", "reconstruct",
-                                        "tpt_argmax", "broadcast", "rope_table"};
+                                        "tpt_argmax", "init_states", "rope_table", "dedup",
+                                        "gather"};
   return (k >= 0 && k < KK_COUNT) ? names[k] : "?";
 }
 

@@ -21,6 +21,8 @@ enum KernelKind {
   KK_TPT,
   KK_BROADCAST,
   KK_ROPE_TABLE,
+  KK_DEDUP,
+  KK_GATHER,
   KK_COUNT
 };
 

@@ -5,9 +5,53 @@
 #include "ks_kernels.cuh"
 
 #include <float.h>
+#include <type_traits>
 #include <math.h>
 
 namespace ks {
+
+// ---------------------------------------------------------------- state hash
+// Order-independent 64-bit fingerprint of a state's fp32 bit patterns: two
+// sums (mod 2^32) of per-element mixes with different keys, so a parallel
+// reduction in any order gives the same value.  fmix32 is the finaliser of
+// MurmurHash3 (Appleby, public domain).  Used only to find states that are
+// bit-for-bit equal; different states collide with probability ~2^-64.
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85ebca6bu;
+  h ^= h >> 13;
+  h *= 0xc2b2ae35u;
+  h ^= h >> 16;
+  return h;
+}
+
+struct Hash2 {
+  uint32_t a = 0, b = 0;
+  __device__ __forceinline__ void add(uint32_t bits, uint32_t idx) {
+    a += fmix32(bits ^ (idx * 0x9e3779b9u));
+    b += fmix32((bits + idx * 0x27d4eb2fu) ^ 0x165667b1u);
+  }
+  __device__ __forceinline__ void add4(float4 v, uint32_t idx4) {
+    add(__float_as_uint(v.x), idx4);
+    add(__float_as_uint(v.y), idx4 + 1);
+    add(__float_as_uint(v.z), idx4 + 2);
+    add(__float_as_uint(v.w), idx4 + 3);
+  }
+};
+
+// Block-wide sum of the fingerprints into *out (one 64-bit word).
+__device__ __forceinline__ void block_hash_store(Hash2 h, uint32_t* sh2, uint64_t* out) {
+  for (int o = 16; o > 0; o >>= 1) {
+    h.a += __shfl_xor_sync(0xffffffffu, h.a, o);
+    h.b += __shfl_xor_sync(0xffffffffu, h.b, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&sh2[0], h.a);
+    atomicAdd(&sh2[1], h.b);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *out = ((uint64_t)sh2[0] << 32) | sh2[1];
+}
 
 // ---------------------------------------------------------------- select
 // One block per budget cell b.  Warps take tokens in turn; each warp sums, in
@@ -138,22 +182,27 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
     float* __restrict__ val, uint8_t* __restrict__ bp, float* __restrict__ cos_s_out,
     float* __restrict__ cos_e_out, float* __restrict__ ref_out,
     const uint8_t* __restrict__ valid_prev, uint8_t* __restrict__ valid_cur, double prune_tau,
-    int min_valid_b) {
+    int min_valid_b, const int* __restrict__ exec_map, uint64_t* __restrict__ hash_cur) {
   __shared__ double cs_tok[kSelectMaxT];
   __shared__ double ce_tok[kSelectMaxT];
   __shared__ float inv_s[kSelectMaxT];
   __shared__ float inv_e[kSelectMaxT];
   __shared__ int take_sh;
+  __shared__ uint32_t hash_sh[2];
   const long long cell = (long long)T * d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_warps = blockDim.x >> 5;
   const int d4 = d / 4;
   const bool is_ref = blockIdx.x == 0;
   const int b = (int)blockIdx.x - 1;
-  const bool has_e = !is_ref && b >= w;
+  // execute candidate: exec slot b - w + 1, or its place in a compacted batch
+  int e_idx = b - w + 1;
+  if (exec_map && !is_ref && b >= w) e_idx = exec_map[b - w + 1];
+  const bool has_e = !is_ref && b >= w && e_idx >= 0;
   // "s" is the skip candidate (or, for the reference slot, the state to keep)
   const float* s_base = is_ref ? exec : prev + (long long)(b + 1) * cell;
-  const float* e_base = has_e ? exec + (long long)(b - w + 1) * cell : nullptr;
+  const float* e_base = has_e ? exec + (long long)e_idx * cell : nullptr;
+  if (threadIdx.x < 2) hash_sh[threadIdx.x] = 0;
   const float* target = target_in ? target_in : exec;
   for (int t = warp; t < T; t += n_warps) {
     const float4* s4 = (const float4*)(s_base + (long long)t * d);
@@ -224,16 +273,19 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
   float4* rdst = (is_ref && ref_out) ? (float4*)ref_out : nullptr;
   TX* xdst = g_next ? xh_next + slot * cell : nullptr;
   const long long n4 = cell / 4;
+  Hash2 hh;
   for (long long i = threadIdx.x; i < n4; i += blockDim.x) {
     const float4 v = src[i];
     dst[i] = v;
     if (rdst) rdst[i] = v;
+    if (hash_cur) hh.add4(v, (uint32_t)(i * 4));
     if (xdst) {
       const int t = (int)(i / d4);
       const int j = (int)(i - (long long)t * d4) * 4;
       store_norm4(xdst + i * 4, v, inv[t], g_next + j);
     }
   }
+  if (hash_cur) block_hash_store(hh, hash_sh, hash_cur + slot);
 }
 
 ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
@@ -241,18 +293,18 @@ ks_status launch_select_fused(const float* prev, const float* exec, const float*
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
                               uint8_t* valid_cur, double prune_tau, int min_valid_b,
-                              cudaStream_t st) {
+                              const int* exec_map, uint64_t* hash_cur, cudaStream_t st) {
   if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "select: T above 256");
   if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "select: d must be a multiple of 4");
   if (wdt == KS_BF16)
     select_fused_kernel<__nv_bfloat16, __nv_bfloat16><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const __nv_bfloat16*)g_next, cur,
         (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out, valid_prev, valid_cur,
-        prune_tau, min_valid_b);
+        prune_tau, min_valid_b, exec_map, hash_cur);
   else
     select_fused_kernel<float, float><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const float*)g_next, cur, (float*)xh_next, val, bp,
-        cos_s, cos_e, ref_out, valid_prev, valid_cur, prune_tau, min_valid_b);
+        cos_s, cos_e, ref_out, valid_prev, valid_cur, prune_tau, min_valid_b, exec_map, hash_cur);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -263,8 +315,11 @@ ks_status launch_select_fused(const float* prev, const float* exec, const float*
 template <typename TX, typename TG>
 __global__ void __launch_bounds__(kSelectThreads) init_states_kernel(
     const float* __restrict__ x0, int T, int d, float eps, const TG* __restrict__ g,
-    float* __restrict__ states, TX* __restrict__ xh, float* __restrict__ ref_out) {
+    float* __restrict__ states, TX* __restrict__ xh, float* __restrict__ ref_out,
+    uint64_t* __restrict__ hash_out) {
   __shared__ float inv_s[kSelectMaxT];
+  __shared__ uint32_t hash_sh[2];
+  if (threadIdx.x < 2) hash_sh[threadIdx.x] = 0;
   const long long cell = (long long)T * d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d4 = d / 4;
@@ -284,26 +339,139 @@ __global__ void __launch_bounds__(kSelectThreads) init_states_kernel(
   float4* dst = (float4*)(states + slot * cell);
   float4* rdst = (slot == 0 && ref_out) ? (float4*)ref_out : nullptr;
   TX* xdst = xh + slot * cell;
+  Hash2 hh;
   for (long long i = threadIdx.x; i < cell / 4; i += blockDim.x) {
     const float4 v = src[i];
     dst[i] = v;
     if (rdst) rdst[i] = v;
+    if (hash_out) hh.add4(v, (uint32_t)(i * 4));
     const int t = (int)(i / d4);
     const int j = (int)(i - (long long)t * d4) * 4;
     store_norm4(xdst + i * 4, v, inv_s[t], g + j);
   }
+  if (hash_out) block_hash_store(hh, hash_sh, hash_out + slot);
 }
 
 ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,
-                             int wdt, float* states, void* xh, float* ref_out, cudaStream_t st) {
+                             int wdt, float* states, void* xh, float* ref_out, uint64_t* hash_out,
+                             cudaStream_t st) {
   if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "init: T above 256");
   if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "init: d must be a multiple of 4");
   if (wdt == KS_BF16)
     init_states_kernel<__nv_bfloat16, __nv_bfloat16><<<n_slots, kSelectThreads, 0, st>>>(
-        x0, T, d, eps, (const __nv_bfloat16*)g, states, (__nv_bfloat16*)xh, ref_out);
+        x0, T, d, eps, (const __nv_bfloat16*)g, states, (__nv_bfloat16*)xh, ref_out, hash_out);
   else
     init_states_kernel<float, float><<<n_slots, kSelectThreads, 0, st>>>(
-        x0, T, d, eps, (const float*)g, states, (float*)xh, ref_out);
+        x0, T, d, eps, (const float*)g, states, (float*)xh, ref_out, hash_out);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+// ---------------------------------------------------------------- distinct-state compaction
+// Slots 0..n-1 of the state buffer (slot 0 = reference, slot s = cell s-1) are
+// the next item's execute sources.  Slots holding bit-identical states (equal
+// fingerprints) and valid are folded onto their first occurrence: map[s] is the
+// compacted index of slot s's state (-1 for an invalid cell), uniq[u] the slot
+// of the u-th distinct state, *count the number of distinct states.  One CTA.
+constexpr int kDedupThreads = 1024;
+constexpr int kDedupMax = 3072;
+
+__global__ void __launch_bounds__(kDedupThreads) dedup_kernel(
+    const uint64_t* __restrict__ hash, const uint8_t* __restrict__ valid, int n,
+    int* __restrict__ map, int* __restrict__ uniq, int* __restrict__ count,
+    int32_t* __restrict__ count_out) {
+  __shared__ uint64_t h[kDedupMax];
+  __shared__ int first[kDedupMax];
+  __shared__ int scan[kDedupThreads];
+  for (int s = threadIdx.x; s < n; s += blockDim.x) h[s] = hash[s];
+  __syncthreads();
+  for (int s = threadIdx.x; s < n; s += blockDim.x) {
+    const bool ok = s == 0 || !valid || valid[s - 1];
+    int f = -1;
+    if (ok) {
+      f = s;
+      for (int q = 0; q < s; ++q) {
+        if (h[q] == h[s] && (q == 0 || !valid || valid[q - 1])) {
+          f = q;
+          break;
+        }
+      }
+    }
+    first[s] = f;
+  }
+  __syncthreads();
+  // exclusive scan of the "first occurrence" flags, each thread owning a run of slots
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  int mine = 0;
+  for (int s = lo; s < hi; ++s) mine += first[s] == s;
+  scan[threadIdx.x] = mine;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+    const int v = threadIdx.x >= (unsigned)off ? scan[threadIdx.x - off] : 0;
+    __syncthreads();
+    scan[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int c = scan[threadIdx.x] - mine;
+  for (int s = lo; s < hi; ++s) {
+    if (first[s] == s) {
+      uniq[c] = s;
+      first[s] = -2 - c;          // remember the compacted index of a first occurrence
+      ++c;
+    }
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < n; s += blockDim.x) {
+    const int f = first[s];
+    map[s] = f == -1 ? -1 : (f <= -2 ? -2 - f : -2 - first[f]);
+  }
+  if (threadIdx.x == blockDim.x - 1) {
+    *count = scan[threadIdx.x];
+    if (count_out) *count_out = scan[threadIdx.x];
+  }
+}
+
+ks_status launch_dedup(const uint64_t* hash, const uint8_t* valid, int n, int* map, int* uniq,
+                       int* count, int32_t* count_out, cudaStream_t st) {
+  if (n > kDedupMax) return fail(KS_ERR_UNSUPPORTED, "dedup: more than 3071 budget cells");
+  dedup_kernel<<<1, kDedupThreads, 0, st>>>(hash, valid, n, map, uniq, count, count_out);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+// Packs the distinct states' fp32 residuals and normalised operands:
+// block u (< *count) copies slot uniq[u] of both buffers to position u.
+template <typename TX>
+__global__ void gather_kernel(const int* __restrict__ uniq, const int* __restrict__ count,
+                              long long cell, const float4* __restrict__ states,
+                              const TX* __restrict__ xh, float4* __restrict__ states_c,
+                              TX* __restrict__ xh_c) {
+  const int u = blockIdx.x;
+  if (u >= *count) return;
+  const long long src = uniq[u];
+  const long long n4 = cell / 4;
+  for (long long i = threadIdx.x; i < n4; i += blockDim.x)
+    states_c[(long long)u * n4 + i] = states[src * n4 + i];
+  // the operand: 8 bytes (bf16) or 16 bytes (fp32) per 4 elements
+  using V = typename std::conditional<sizeof(TX) == 2, uint2, float4>::type;
+  const V* xs = reinterpret_cast<const V*>(xh + src * cell);
+  V* xd = reinterpret_cast<V*>(xh_c + (long long)u * cell);
+  for (long long i = threadIdx.x; i < n4; i += blockDim.x) xd[i] = xs[i];
+}
+
+ks_status launch_gather(const int* uniq, const int* count, int max_count, long long cell,
+                        const float* states, const void* xh, int act, float* states_c, void* xh_c,
+                        cudaStream_t st) {
+  if (cell % 4) return fail(KS_ERR_UNSUPPORTED, "gather: T*d must be a multiple of 4");
+  if (act == ACT_BF16)
+    gather_kernel<__nv_bfloat16><<<max_count, 512, 0, st>>>(
+        uniq, count, cell, (const float4*)states, (const __nv_bfloat16*)xh, (float4*)states_c,
+        (__nv_bfloat16*)xh_c);
+  else
+    gather_kernel<float><<<max_count, 512, 0, st>>>(uniq, count, cell, (const float4*)states,
+                                                    (const float*)xh, (float4*)states_c,
+                                                    (float*)xh_c);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -359,6 +527,14 @@ ks_status launch_reconstruct(const uint8_t* bp, const int32_t* w, const double* 
   const ItemTable& tb = tab ? *tab : empty;
   reconstruct_kernel<<<ceil_div(C, 128), 128, 0, st>>>(bp, w, t, tb, tab != nullptr, n_items, C,
                                                        sets, used_w, t_draft, status, valid);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+__global__ void fill_i32_kernel(int32_t* p, int32_t v) { *p = v; }
+
+ks_status launch_fill_i32(int32_t* p, int32_t v, cudaStream_t st) {
+  fill_i32_kernel<<<1, 1, 0, st>>>(p, v);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }

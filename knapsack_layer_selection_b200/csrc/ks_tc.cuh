@@ -22,9 +22,11 @@ bool use_tensor_cores(const ks_model_desc* m);
 // A [M][K], B/B2 [N][K] bf16 row-major; K a multiple of 64; N a multiple of 256
 // (128 for SwiGLU, whose output has N columns).  status: device word for a
 // bounded-wait timeout, or NULL.
+// dyn_cells (device int, optional): only the first *dyn_cells x T rows are live
+// (a batch compacted on the device); M is then an upper bound.
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
-                  int32_t* status, cudaStream_t st);
+                  int32_t* status, cudaStream_t st, const int* dyn_cells = nullptr);
 
 // Tensor map of a row-major bf16 matrix [rows][cols] (row_stride elements apart)
 // read in boxes of box_rows x box_cols with the 128-byte swizzle; reads outside
@@ -37,7 +39,7 @@ ks_status make_tmap_2d(CUtensorMap* m, const void* base, long long rows, long lo
 // bf16; token t attends to positions 0 .. ctx + t.  hd = 64 or 128.
 ks_status tc_attention(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
                        int T, int Hq, int Hkv, int hd, int ctx, void* out, int32_t* status,
-                       cudaStream_t st);
+                       cudaStream_t st, const int* dyn_cells = nullptr);
 
 int sm_count();
 

@@ -83,6 +83,7 @@ struct AttnParams {
   int32_t* status;
   int R, T, Hq, Hkv, ctx, n_keys, n_blocks;
   float scale_log2;
+  const int* dyn_cells;   // optional device count: R = min(R, *dyn_cells * T) at run time
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -183,8 +184,14 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 template <int HD>
 __global__ void __launch_bounds__(320, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p_in) {
   using C = Cfg<HD>;
+  AttnParams p = p_in;
+  if (p.dyn_cells) {
+    const long long live = (long long)(*p.dyn_cells) * p.T;
+    p.R = (int)(live < p.R ? live : p.R);
+  }
+  if ((int)blockIdx.x * C::BM >= p.R) return;   // a row tile past the live rows: nothing to do
   extern __shared__ __align__(1024) unsigned char smem[];
   // the 128-byte-swizzled tiles need a 1024-aligned base; the layout uses all of
   // shared memory, so there is no room to realign -- refuse instead
@@ -512,7 +519,7 @@ __global__ void __launch_bounds__(320, 1)
 template <int HD>
 ks_status launch_attn(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
                       int T, int Hq, int Hkv, int ctx, void* out, int32_t* status,
-                      cudaStream_t st) {
+                      cudaStream_t st, const int* dyn_cells) {
   using C = Cfg<HD>;
   static bool attr = false;
   auto k = attn_kernel<HD>;
@@ -537,6 +544,7 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, long long c
   ap.n_keys = n_keys;
   ap.n_blocks = (n_keys + C::BN - 1) / C::BN;
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
+  ap.dyn_cells = dyn_cells;
   dim3 grid((R + C::BM - 1) / C::BM, Hq);
   k<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, ap);
   KS_LAUNCH_CHECK();
@@ -547,12 +555,14 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, long long c
 
 ks_status tc_attention(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
                        int T, int Hq, int Hkv, int hd, int ctx, void* out, int32_t* status,
-                       cudaStream_t st) {
+                       cudaStream_t st, const int* dyn_cells) {
   if (R <= 0) return KS_OK;
   if (Hq % Hkv) return fail(KS_ERR_INVALID_ARG, "attention: Hq must be a multiple of Hkv");
   if (cache_rows < (long long)ctx + T) return fail(KS_ERR_INVALID_ARG, "attention: cache too short");
-  if (hd == 128) return launch_attn<128>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st);
-  if (hd == 64) return launch_attn<64>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st);
+  if (hd == 128)
+    return launch_attn<128>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
+  if (hd == 64)
+    return launch_attn<64>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
   return fail(KS_ERR_UNSUPPORTED, "attention: head_dim must be 64 or 128");
 }
 

@@ -75,6 +75,7 @@ struct GemmParams {
   int tiles_m, tiles_n;
   int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
   int T, head_dim;
+  const int* dyn_cells; // optional device count: M = min(M, *dyn_cells * T) at run time
 };
 
 // Tile t of the walk -> (m-tile, n-tile).  Tiles go in groups of group_m m-tiles;
@@ -93,7 +94,15 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm,
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmB2, const GemmParams p_in) {
+  // rows can be decided on the device (a compacted batch): the walk uses the live count
+  GemmParams p = p_in;
+  if (p.dyn_cells) {
+    const long long live = (long long)(*p.dyn_cells) * p.T;
+    p.M = (int)(live < p.M ? live : p.M);
+    p.tiles_m = (p.M + BM - 1) / BM;
+    if (p.group_m > p.tiles_m) p.group_m = p.tiles_m > 0 ? p.tiles_m : 1;
+  }
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   SharedTail* tail = reinterpret_cast<SharedTail*>(smem + STAGES * STAGE_BYTES);
@@ -360,7 +369,7 @@ bool use_tensor_cores(const ks_model_desc* m) { return m->wdtype == KS_BF16; }
 
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
-                  int32_t* status, cudaStream_t st) {
+                  int32_t* status, cudaStream_t st, const int* dyn_cells) {
   if (M <= 0) return KS_OK;
   if (K % BK) return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: K must be a multiple of 64");
   const int bn_out = epi == EPI_SWIGLU_BF16 ? BN / 2 : BN;
@@ -400,6 +409,7 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
   }
   gp.T = T;
   gp.head_dim = head_dim;
+  gp.dyn_cells = dyn_cells;
   switch (epi) {
     case EPI_RESID_F32: return launch<EPI_RESID_F32>(ta, tb, tb2, gp, st);
     case EPI_ROPE_BF16: return launch<EPI_ROPE_BF16>(ta, tb, tb2, gp, st);
