@@ -116,6 +116,28 @@ def test_full_size_solve(name):
     rep.assert_ok()
 
 
+def test_full_size_dedup_is_bit_identical():
+    """Distinct-state execution at the 8B shape reproduces the dense solve."""
+    wl = W.WORKLOADS["llama3_8b_8k"]
+    inp = W.make_inputs(wl)
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    outs = []
+    for dd in (False, True):
+        s = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, wl.latencies(),
+                     B.params(wl.gamma_max, wl.n_bins, dedup=dd))
+        s.solve(inp.x0)
+        torch.cuda.synchronize()
+        s.check_status()
+        outs.append((s, {k: getattr(s.out, k).cpu().numpy() for k in
+                         ("bp", "values", "sets", "best", "ref_states", "exec_counts")}))
+    (sd, d), (sq, q) = outs
+    for k in ("bp", "values", "sets", "best", "ref_states"):
+        assert np.array_equal(d[k], q[k]), k
+    print(f"\n8B @ 8k: distinct states executed {int(q['exec_counts'].sum())} of "
+          f"{int(d['exec_counts'].sum())}")
+
+
 def test_long_context_resolve_shifts_the_layer_set():
     """Re-solve the 8B shape at 4k, 16k and 32k context (the 64-step re-solve of
     the paper's serving loop, done here at three contexts): report how the
