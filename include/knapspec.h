@@ -159,6 +159,7 @@ typedef struct {
                           the solve computed (they ride along in each item's batch) */
   int32_t* exec_counts; /* [n_items] optional: states item k ran on (with dedup: the
                            distinct ones, the reference included) */
+  float* final_states;  /* [C][T][d] optional: every cell's state after the last item */
 } ks_result;
 
 /* Library version string (static storage). */
@@ -343,6 +344,36 @@ KS_API ks_status ks_solve_cells(int32_t n_items, const int32_t* w, const double*
  */
 KS_API ks_status ks_check_bounded_wait(uint32_t limit_us, int32_t* status, uint64_t* waited_ns,
                                        ks_stream_t stream);
+
+/*
+ * Lemma 4.1 checker (review page: §4 Lemma 4.1, referee major 2, "What would
+ * settle it").  For N states [N][T][d] (e.g. ks_result.final_states) and the
+ * full model's final state ref [T][d] (ks_result.ref_states row n_items):
+ * h = RMSNorm(ref_t) * g, h' = RMSNorm(state_t) * g rescaled to ||h|| (equal
+ * norms, the lemma's premise), logits through lm_head W [V][d] bf16:
+ * i*_t = argmax W h (first on ties), margin_t = z_i* - max_{j != i*} z_j,
+ * dist_t = max_j ||w_i* - w_j||.  bound[n][t] = (||h - h'|| * dist < margin),
+ * the lemma's sufficient condition for argmax W h' = i*; agree[n][t] = (argmax
+ * W h' = i*).  counts = {#bound, #agree, #bound-and-not-agree}.  Operands of
+ * the logits are rounded to bf16 (fp32 accumulation); the norms and cosines
+ * are fp64 sums.  final_norm: bf16 [d] gain or NULL (gain 1).  d a multiple of
+ * 64, V of 256.  All buffers are device memory.
+ */
+typedef struct {
+  int32_t* istar;      /* [T] */
+  float* margin;       /* [T] */
+  float* dist;         /* [T] */
+  float* cos;          /* [N][T] cosine of h' with h */
+  uint8_t* bound;      /* [N][T] */
+  uint8_t* agree;      /* [N][T] */
+  int32_t* counts;     /* [3] */
+} ks_lemma_result;
+
+KS_API ks_status ks_lemma_workspace_size(int32_t N, int32_t T, int32_t d, int32_t V, size_t* bytes);
+KS_API ks_status ks_lemma_check(const float* states, int32_t N, const float* ref, int32_t T,
+                                int32_t d, const void* final_norm, float eps, const void* lm_head,
+                                int32_t V, void* workspace, size_t workspace_bytes,
+                                ks_lemma_result* out, int32_t* status, ks_stream_t stream);
 
 /*
  * Launch accounting.  Between ks_profile_start and ks_profile_stop the library

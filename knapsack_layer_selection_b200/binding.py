@@ -56,7 +56,8 @@ class Params(ctypes.Structure):
 class Result(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("status", "values", "sets", "used_w", "t_draft", "bp", "cos_skip",
-                 "cos_exec", "tpt", "best", "best_tpt", "ref_states", "exec_counts")]
+                 "cos_exec", "tpt", "best", "best_tpt", "ref_states", "exec_counts",
+                 "final_states")]
 
 
 class KernelStat(ctypes.Structure):
@@ -70,7 +71,7 @@ EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weigh
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
            "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
            "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16",
-           "ks_check_bounded_wait"]
+           "ks_check_bounded_wait", "ks_lemma_workspace_size", "ks_lemma_check"]
 
 _lib = None
 
@@ -103,6 +104,9 @@ def load() -> ctypes.CDLL:
         "ks_workspace_status": ([P, ctypes.POINTER(I32), P], ctypes.c_int),
         "ks_gemm_bf16": ([P, P, P, P, I32, I32, I32, P, P], ctypes.c_int),
         "ks_check_bounded_wait": ([ctypes.c_uint32, P, P, P], ctypes.c_int),
+        "ks_lemma_workspace_size": ([I32, I32, I32, I32, ctypes.POINTER(SZ)], ctypes.c_int),
+        "ks_lemma_check": ([P, I32, P, I32, I32, P, ctypes.c_float, P, I32, P, SZ, P, P, P],
+                           ctypes.c_int),
         "ks_attention_bf16": ([P, P, P, I64, I32, I32, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
     }
@@ -312,6 +316,7 @@ class SolveOutputs:
     tpt: Optional[torch.Tensor] = None
     ref_states: Optional[torch.Tensor] = None
     exec_counts: Optional[torch.Tensor] = None
+    final_states: Optional[torch.Tensor] = None
 
 
 class Solver:
@@ -321,7 +326,7 @@ class Solver:
                  k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int, T: int,
                  t: Sequence[float], prm: Params, w: Optional[Sequence[int]] = None,
                  keep_bp: bool = True, keep_cos: bool = False, keep_tpt: bool = True,
-                 keep_ref: bool = True, device="cuda"):
+                 keep_ref: bool = True, keep_final: bool = False, device="cuda"):
         self.model = model
         self.wdtype = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
         self._layers_keep = layers
@@ -349,12 +354,14 @@ class Solver:
             cos_exec=z(n, C, dt=torch.float32) if keep_cos else None,
             tpt=z(C, prm.gamma_max, dt=torch.float64) if keep_tpt else None,
             ref_states=z(n + 1, T, model.d_model, dt=torch.float32) if keep_ref else None,
-            exec_counts=z(n, dt=torch.int32))
+            exec_counts=z(n, dt=torch.int32),
+            final_states=z(C, T, model.d_model, dt=torch.float32) if keep_final else None)
         o = self.out
         p = lambda x: None if x is None else x.data_ptr()
         self.result = Result(p(o.status), p(o.values), p(o.sets), p(o.used_w), p(o.t_draft),
                              p(o.bp), p(o.cos_skip), p(o.cos_exec), p(o.tpt), p(o.best),
-                             p(o.best_tpt), p(o.ref_states), p(o.exec_counts))
+                             p(o.best_tpt), p(o.ref_states), p(o.exec_counts),
+                             p(o.final_states))
         self._t_arr = (ctypes.c_double * n)(*self.t)
         self._w_arr = (ctypes.c_int32 * n)(*self.w)
 
@@ -386,6 +393,40 @@ def profile_stop() -> List[dict]:
     return [{"name": arr[i].name.decode(), "launches": arr[i].launches,
              "total_ms": arr[i].total_ms, "flops": arr[i].flops, "bytes": arr[i].bytes}
             for i in range(min(n.value, 64))]
+
+
+class LemmaResult(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("istar", "margin", "dist", "cos", "bound", "agree", "counts")]
+
+
+def lemma_check(states: torch.Tensor, ref: torch.Tensor, lm_head: torch.Tensor,
+                final_norm: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                status: Optional[torch.Tensor] = None) -> dict:
+    """Lemma 4.1 checker on N states [N][T][d] against ref [T][d] (see knapspec.h)."""
+    N, T, d = states.shape
+    V = lm_head.shape[0]
+    size = ctypes.c_size_t()
+    _check(load().ks_lemma_workspace_size(N, T, d, V, ctypes.byref(size)))
+    ws = torch.empty(size.value, dtype=torch.uint8, device=states.device)
+    dev = states.device
+    out = {"istar": torch.empty(T, dtype=torch.int32, device=dev),
+           "margin": torch.empty(T, dtype=torch.float32, device=dev),
+           "dist": torch.empty(T, dtype=torch.float32, device=dev),
+           "cos": torch.empty(N, T, dtype=torch.float32, device=dev),
+           "bound": torch.empty(N, T, dtype=torch.uint8, device=dev),
+           "agree": torch.empty(N, T, dtype=torch.uint8, device=dev),
+           "counts": torch.empty(3, dtype=torch.int32, device=dev)}
+    res = LemmaResult(*[out[k].data_ptr() for k in
+                        ("istar", "margin", "dist", "cos", "bound", "agree", "counts")])
+    _check(load().ks_lemma_check(_dev(states, torch.float32, "states"), N,
+                                 _dev(ref, torch.float32, "ref"), T, d,
+                                 _dev(final_norm, torch.bfloat16, "final_norm"), eps,
+                                 _dev(lm_head, torch.bfloat16, "lm_head"), V, ws.data_ptr(),
+                                 ws.numel(), ctypes.byref(res), _dev(status, torch.int32, "status"),
+                                 _stream()))
+    out["_ws"] = ws
+    return out
 
 
 def sets_to_lists(sets: torch.Tensor, n_items: int) -> List[List[int]]:

@@ -569,6 +569,9 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     std::swap(vprev, vcur);
     std::swap(hprev, hcur);
   }
+  if (out->final_states)
+    KS_CUDA_TRY(cudaMemcpyAsync(out->final_states, prev + cell, (size_t)C * cell * sizeof(float),
+                                cudaMemcpyDeviceToDevice, st));
   double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;
   {
     ProfScope ps(KK_RECONSTRUCT, st, 0.0, (double)n_items * C);

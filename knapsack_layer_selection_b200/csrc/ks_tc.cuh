@@ -14,6 +14,14 @@ enum Epilogue {
   EPI_SWIGLU_BF16 = 2,  // out bf16 [M][N] = silu(A.Bg^T) * (A.Bu^T)  (B = gate, B2 = up)
   EPI_STORE_BF16 = 3,   // out bf16 [M][N] = acc
   EPI_STORE_F32 = 4,    // out fp32 [M][N] = acc
+  EPI_ROWMAX = 5,       // out float4 [M][N/256]: per row and 256-column tile, of
+                        // v = scale * acc + col_bias[n]: {top-1, index (int bits), top-2, 0}
+};
+
+// Parameters of the row-maximum epilogue (EPI_ROWMAX).
+struct RowMaxArgs {
+  float scale;
+  const float* col_bias;   // [N] or NULL
 };
 
 // True when the model's contractions run on the tensor cores (bf16 weights).
@@ -26,7 +34,8 @@ bool use_tensor_cores(const ks_model_desc* m);
 // (a batch compacted on the device); M is then an upper bound.
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
-                  int32_t* status, cudaStream_t st, const int* dyn_cells = nullptr);
+                  int32_t* status, cudaStream_t st, const int* dyn_cells = nullptr,
+                  RowMaxArgs rowmax = RowMaxArgs{1.0f, nullptr});
 
 // Tensor map of a row-major bf16 matrix [rows][cols] (row_stride elements apart)
 // read in boxes of box_rows x box_cols with the 128-byte swizzle; reads outside

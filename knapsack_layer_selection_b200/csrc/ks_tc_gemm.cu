@@ -76,6 +76,7 @@ struct GemmParams {
   int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
   int T, head_dim;
   const int* dyn_cells; // optional device count: M = min(M, *dyn_cells * T) at run time
+  RowMaxArgs rowmax;    // EPI_ROWMAX only
 };
 
 // Tile t of the walk -> (m-tile, n-tile).  Tiles go in groups of group_m m-tiles;
@@ -250,6 +251,31 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
+      } else if (EPI == EPI_ROWMAX) {
+        // top-2 of scale * acc + bias over this tile's 256 columns of the row
+        const int n0 = tn * BN;
+        float v1 = -INFINITY, v2 = -INFINITY;
+        int i1 = -1;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = n0 + c * 32 + j;
+            const float x = p.rowmax.scale * v[j] + (p.rowmax.col_bias ? p.rowmax.col_bias[col] : 0.f);
+            if (x > v1) {
+              v2 = v1;
+              v1 = x;
+              i1 = col;
+            } else if (x > v2) {
+              v2 = x;
+            }
+          }
+        }
+        if (live)
+          reinterpret_cast<float4*>(p.out)[(long long)row * p.tiles_n + tn] =
+              make_float4(v1, __int_as_float(i1), v2, 0.f);
       } else if (EPI == EPI_SWIGLU_BF16) {
         // columns 0..127: gate, 128..255: up, for output columns tn*128 ..
         const int n0 = tn * (BN / 2);
@@ -369,7 +395,7 @@ bool use_tensor_cores(const ks_model_desc* m) { return m->wdtype == KS_BF16; }
 
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
-                  int32_t* status, cudaStream_t st, const int* dyn_cells) {
+                  int32_t* status, cudaStream_t st, const int* dyn_cells, RowMaxArgs rowmax) {
   if (M <= 0) return KS_OK;
   if (K % BK) return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: K must be a multiple of 64");
   const int bn_out = epi == EPI_SWIGLU_BF16 ? BN / 2 : BN;
@@ -410,12 +436,14 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
   gp.T = T;
   gp.head_dim = head_dim;
   gp.dyn_cells = dyn_cells;
+  gp.rowmax = rowmax;
   switch (epi) {
     case EPI_RESID_F32: return launch<EPI_RESID_F32>(ta, tb, tb2, gp, st);
     case EPI_ROPE_BF16: return launch<EPI_ROPE_BF16>(ta, tb, tb2, gp, st);
     case EPI_SWIGLU_BF16: return launch<EPI_SWIGLU_BF16>(ta, tb, tb2, gp, st);
     case EPI_STORE_BF16: return launch<EPI_STORE_BF16>(ta, tb, tb2, gp, st);
     case EPI_STORE_F32: return launch<EPI_STORE_F32>(ta, tb, tb2, gp, st);
+    case EPI_ROWMAX: return launch<EPI_ROWMAX>(ta, tb, tb2, gp, st);
   }
   return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: unknown epilogue");
 }

@@ -195,6 +195,22 @@ def truncated(wl: Workload, n_layers: int, ctx: Optional[int] = None) -> Workloa
     return dataclasses.replace(wl, n_layers=n_layers, ctx=wl.ctx if ctx is None else ctx)
 
 
+# Vocabulary sizes of the synthetic LM heads used by the Lemma 4.1 checker
+# (the 8B and 32B shapes use Llama-3's and a 256-aligned Qwen3-like size).
+VOCAB = {"tiny": 1024, "small": 8192, "llama3_8b_8k": 128256, "llama3_8b_32k": 128256,
+         "qwen3_32b_16k": 151808}
+
+
+def lm_head(wl: Workload, seed: int = 1, device: Optional[str] = None,
+            vocab: Optional[int] = None) -> torch.Tensor:
+    """A random LM head W [V][d] ~ N(0, 0.02^2) in bf16 (its own generator and seed)."""
+    dev = device or wl.gen_device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    V = vocab or VOCAB[wl.name]
+    return _randn((V, wl.d_model), LINEAR_STD, torch.bfloat16, gen, dev)
+
+
 def random_states(shape: Sequence[int], seed: int, device: str = "cpu",
                   dtype: torch.dtype = torch.float32) -> torch.Tensor:
     """N(0,1) tensor of the given shape (for kernel-level tests of one step)."""

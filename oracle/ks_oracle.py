@@ -573,3 +573,53 @@ def scalar_knapsack_dp(w: Sequence[int], v: Sequence[int], capacity: int,
                       prune=pruning_rule(w, C, prune_tau, skip_cap))
     vals = np.where(res.valid[len(w)], res.val[len(w)], -np.inf)
     return vals, res
+
+
+# --------------------------------------------------------------------------
+# Lemma 4.1 checker: does cosine closeness guarantee the same greedy token?
+# --------------------------------------------------------------------------
+@dataclass
+class LemmaCheck:
+    istar: np.ndarray      # [T] greedy token of the reference state
+    margin: np.ndarray     # [T] xi = z_i* - max_{j != i*} z_j
+    dist: np.ndarray       # [T] D = max_j ||w_i* - w_j||
+    cos: np.ndarray        # [N, T] cosine of each state's token with the reference token
+    bound: np.ndarray      # [N, T] the sufficient condition ||h - h'|| < xi / D holds
+    agree: np.ndarray      # [N, T] argmax W h' == i*
+    state_margin: np.ndarray   # [N, T] top-1 minus top-2 logit of h'
+    slack: np.ndarray      # [N, T] xi / D - ||h - h'||
+
+
+def lemma_check(states: np.ndarray, ref: np.ndarray, lm_head: np.ndarray,
+                final_gain: Optional[np.ndarray], eps: float) -> LemmaCheck:
+    """The review's Lemma 4.1 (KnapSpec §4, referee major 2 and "What carries the
+    argument") evaluated on DP states.
+
+    h = RMSNorm(ref_t) and h' = RMSNorm(state_t) rescaled to ||h|| (the lemma's
+    equal-norm premise).  With logits z = W h, i* = argmax z, margin
+    xi = z_i* - max_{j != i*} z_j and D = max_j ||w_i* - w_j||, the lemma says
+    ||h - h'|| < xi / D implies argmax W h' = i*: for every j,
+    (w_i* - w_j).h' >= (w_i* - w_j).h - ||w_i* - w_j|| ||h' - h|| >= xi - D ||h' - h|| > 0
+    (Cauchy-Schwarz).  Equal norms give ||h - h'||^2 = 2 ||h||^2 (1 - cos).
+    """
+    W = np.asarray(lm_head, F64)
+    S = np.asarray(states, F64)
+    R = np.asarray(ref, F64)
+    g = np.ones(R.shape[-1]) if final_gain is None else np.asarray(final_gain, F64)
+    h = rms_norm(R, g, eps)                          # [T, d]
+    hp = rms_norm(S, g, eps)                         # [N, T, d]
+    nh = np.linalg.norm(h, axis=-1)                  # [T]
+    hp = hp * (nh / np.linalg.norm(hp, axis=-1))[..., None]
+    z = h @ W.T                                      # [T, V]
+    istar = np.argmax(z, axis=-1)
+    top = np.sort(z, axis=-1)
+    margin = top[:, -1] - top[:, -2]
+    dist = np.array([np.max(np.linalg.norm(W - W[i], axis=-1)) for i in istar])
+    cos = np.sum(hp * h[None], axis=-1) / (nh[None] * nh[None])
+    gap = np.sqrt(np.maximum(2.0 * nh[None] ** 2 * (1.0 - cos), 0.0))   # ||h - h'||
+    slack = margin[None] / dist[None] - gap
+    zp = hp @ W.T                                    # [N, T, V]
+    agree = np.argmax(zp, axis=-1) == istar[None]
+    tp = np.sort(zp, axis=-1)
+    return LemmaCheck(istar=istar, margin=margin, dist=dist, cos=cos, bound=slack > 0,
+                      agree=agree, state_margin=tp[..., -1] - tp[..., -2], slack=slack)

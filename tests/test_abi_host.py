@@ -124,7 +124,7 @@ def test_solve_rejects_null_and_short_workspace_before_any_launch(lib):
     for f, _ in B.LayerWeights._fields_:
         setattr(layers[0], f, 256)
     cache = B.CacheDesc(256, 256, 16, 8)
-    res = B.Result(*([256] * 13))
+    res = B.Result(*([256] * 14))
     st = lib.ks_solve(ctypes.byref(m), layers, ctypes.byref(cache), 4, x0, None, None, t,
                       ctypes.byref(prm), ctypes.c_void_p(256), 1024, ctypes.byref(res), None)
     assert st == 3 and b"workspace" in lib.ks_last_error()
@@ -140,7 +140,7 @@ def test_solve_rejects_unknown_budget_mode(lib):
     prm = B.params(4, 8)
     prm.budget_mode = 7
     t = (ctypes.c_double * 2)(1.0, 1.0)
-    res = B.Result(*([256] * 13))
+    res = B.Result(*([256] * 14))
     st = lib.ks_solve(ctypes.byref(m), None, None, 4, ctypes.c_void_p(256), None, None, t,
                       ctypes.byref(prm), None, 0, ctypes.byref(res), None)
     assert st == 1 and b"budget_mode" in lib.ks_last_error()

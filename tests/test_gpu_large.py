@@ -138,6 +138,29 @@ def test_full_size_dedup_is_bit_identical():
           f"{int(d['exec_counts'].sum())}")
 
 
+def test_full_size_lemma_measurement():
+    """Lemma 4.1 on the 8B shape's final DP states with a random LM head of Llama-3's
+    vocabulary: how often the sufficient condition holds vs greedy agreement."""
+    wl = W.WORKLOADS["llama3_8b_8k"]
+    inp = W.make_inputs(wl)
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    s = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, wl.latencies(),
+                 B.params(wl.gamma_max, wl.n_bins, dedup=True), keep_final=True)
+    s.solve(inp.x0)
+    torch.cuda.synchronize()
+    s.check_status()
+    head = W.lm_head(wl)
+    res = B.lemma_check(s.out.final_states, s.out.ref_states[-1].contiguous(), head)
+    torch.cuda.synchronize()
+    c = res["counts"].cpu().tolist()
+    n = s.C * wl.T
+    assert c[2] == 0 or c[2] <= max(1, n // 1000)   # only rounding-level exceptions
+    assert bool(res["agree"][-1].all())
+    print(f"\n8B @ 8k, V={head.shape[0]}: bound holds {c[0]}/{n}, greedy agrees {c[1]}/{n}, "
+          f"bound without agreement {c[2]}")
+
+
 def test_long_context_resolve_shifts_the_layer_set():
     """Re-solve the 8B shape at 4k, 16k and 32k context (the 64-step re-solve of
     the paper's serving loop, done here at three contexts): report how the

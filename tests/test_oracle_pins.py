@@ -479,3 +479,61 @@ def test_disabled_rules_change_nothing(tiny, tiny_solve):
     p = O.dp_solve(m, x0_np(inp), wl.ctx, s.w, s.t, wl.gamma_max, per_cell=True,
                    prune_tau=-np.inf, skip_cap=sum(s.w))
     assert np.array_equal(p.dp.bp, s.dp.bp) and np.array_equal(p.values, s.values)
+
+
+# ---------------------------------------------------------------- Lemma 4.1 checker
+def _lemma_case(seed, N=6, T=5, d=48, V=40):
+    rng = np.random.default_rng(seed)
+    W = rng.normal(0, 1, (V, d))
+    ref = rng.normal(0, 1, (T, d))
+    states = ref[None] + rng.normal(0, 1, (N, T, d)) * rng.uniform(0.001, 0.6, (N, 1, 1))
+    return states, ref, W
+
+
+def test_lemma_margin_and_distance_by_brute_force():
+    states, ref, W = _lemma_case(0)
+    lc = O.lemma_check(states, ref, W, None, 1e-6)
+    for t in range(ref.shape[0]):
+        h = ref[t] / np.sqrt(np.mean(ref[t] ** 2) + 1e-6)
+        z = [float(W[j] @ h) for j in range(W.shape[0])]
+        i = max(range(len(z)), key=lambda j: z[j])
+        assert lc.istar[t] == i
+        assert abs(lc.margin[t] - (z[i] - max(z[j] for j in range(len(z)) if j != i))) < 1e-12
+        D = max(math.sqrt(sum((W[i][c] - W[j][c]) ** 2 for c in range(W.shape[1])))
+                for j in range(W.shape[0]))
+        assert abs(lc.dist[t] - D) < 1e-12
+
+
+def test_lemma_equal_norm_distance_identity():
+    states, ref, W = _lemma_case(1)
+    lc = O.lemma_check(states, ref, W, None, 1e-6)
+    h = ref / np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True) + 1e-6)
+    hp = states / np.sqrt(np.mean(states ** 2, axis=-1, keepdims=True) + 1e-6)
+    hp = hp * (np.linalg.norm(h, axis=-1) / np.linalg.norm(hp, axis=-1))[..., None]
+    gap = np.linalg.norm(hp - h[None], axis=-1)
+    assert np.allclose(gap, lc.margin[None] / lc.dist[None] - lc.slack, atol=1e-9)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_lemma_bound_implies_agreement_even_at_the_boundary(seed):
+    """The sufficient condition never fails: random states, plus states pushed
+    to 0.999 of the allowed distance along the most harmful direction."""
+    states, ref, W = _lemma_case(seed)
+    lc = O.lemma_check(states, ref, W, None, 1e-6)
+    assert not np.any(lc.bound & ~lc.agree)
+    # adversarial: move h toward w_j - w_i* (the runner-up's direction) by 0.999 xi / D
+    T, d = ref.shape
+    h = ref / np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True) + 1e-6)
+    adv = []
+    for t in range(T):
+        i = lc.istar[t]
+        z = W @ h[t]
+        j = np.argsort(z)[-2]
+        u = W[j] - W[i]
+        u -= (u @ h[t]) / (h[t] @ h[t]) * h[t]          # tangent direction keeps the norm to 1st order
+        u /= np.linalg.norm(u)
+        r = 0.999 * lc.margin[t] / lc.dist[t]
+        adv.append(h[t] + r * u)
+    adv = np.array(adv)[None]
+    lc2 = O.lemma_check(adv, ref, W, None, 1e-6)
+    assert not np.any(lc2.bound & ~lc2.agree)
