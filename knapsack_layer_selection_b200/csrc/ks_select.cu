@@ -204,22 +204,38 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
   const float* e_base = has_e ? exec + (long long)e_idx * cell : nullptr;
   if (threadIdx.x < 2) hash_sh[threadIdx.x] = 0;
   const float* target = target_in ? target_in : exec;
+  constexpr int U = 4;   // loads issued ahead per lane: keeps enough bytes in flight for HBM
   for (int t = warp; t < T; t += n_warps) {
     const float4* s4 = (const float4*)(s_base + (long long)t * d);
     const float4* r4 = (const float4*)(target + (long long)t * d);
     const float4* e4 = has_e ? (const float4*)(e_base + (long long)t * d) : nullptr;
     double sr = 0, ss = 0, rr = 0, er = 0, ee = 0;
-    for (int i = lane; i < d4; i += 32) {
-      const float4 sv = s4[i];
-      ss += (double)sv.x * sv.x + (double)sv.y * sv.y + (double)sv.z * sv.z + (double)sv.w * sv.w;
-      if (!is_ref) {
-        const float4 r = r4[i];
-        sr += (double)sv.x * r.x + (double)sv.y * r.y + (double)sv.z * r.z + (double)sv.w * r.w;
-        rr += (double)r.x * r.x + (double)r.y * r.y + (double)r.z * r.z + (double)r.w * r.w;
-        if (has_e) {
-          const float4 e = e4[i];
-          er += (double)e.x * r.x + (double)e.y * r.y + (double)e.z * r.z + (double)e.w * r.w;
-          ee += (double)e.x * e.x + (double)e.y * e.y + (double)e.z * e.z + (double)e.w * e.w;
+    for (int i0 = lane; i0 < d4; i0 += 32 * U) {
+      float4 sv[U], rv[U], ev[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < d4) {
+          sv[u] = s4[i];
+          if (!is_ref) rv[u] = r4[i];
+          if (has_e) ev[u] = e4[i];
+        }
+      }
+      // accumulate in increasing i, the same order for every slot
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (i0 + 32 * u >= d4) break;
+        const float4 a = sv[u];
+        ss += (double)a.x * a.x + (double)a.y * a.y + (double)a.z * a.z + (double)a.w * a.w;
+        if (!is_ref) {
+          const float4 r = rv[u];
+          sr += (double)a.x * r.x + (double)a.y * r.y + (double)a.z * r.z + (double)a.w * r.w;
+          rr += (double)r.x * r.x + (double)r.y * r.y + (double)r.z * r.z + (double)r.w * r.w;
+          if (has_e) {
+            const float4 e = ev[u];
+            er += (double)e.x * r.x + (double)e.y * r.y + (double)e.z * r.z + (double)e.w * r.w;
+            ee += (double)e.x * e.x + (double)e.y * e.y + (double)e.z * e.z + (double)e.w * e.w;
+          }
         }
       }
     }
@@ -274,15 +290,26 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
   TX* xdst = g_next ? xh_next + slot * cell : nullptr;
   const long long n4 = cell / 4;
   Hash2 hh;
-  for (long long i = threadIdx.x; i < n4; i += blockDim.x) {
-    const float4 v = src[i];
-    dst[i] = v;
-    if (rdst) rdst[i] = v;
-    if (hash_cur) hh.add4(v, (uint32_t)(i * 4));
-    if (xdst) {
-      const int t = (int)(i / d4);
-      const int j = (int)(i - (long long)t * d4) * 4;
-      store_norm4(xdst + i * 4, v, inv[t], g_next + j);
+  for (long long i0 = threadIdx.x; i0 < n4; i0 += (long long)blockDim.x * U) {
+    float4 vv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + (long long)u * blockDim.x;
+      if (i < n4) vv[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + (long long)u * blockDim.x;
+      if (i >= n4) break;
+      const float4 v = vv[u];
+      dst[i] = v;
+      if (rdst) rdst[i] = v;
+      if (hash_cur) hh.add4(v, (uint32_t)(i * 4));
+      if (xdst) {
+        const int t = (int)(i / d4);
+        const int j = (int)(i - (long long)t * d4) * 4;
+        store_norm4(xdst + i * 4, v, inv[t], g_next + j);
+      }
     }
   }
   if (hash_cur) block_hash_store(hh, hash_sh, hash_cur + slot);
