@@ -1,10 +1,13 @@
 """A small, self-contained case for profiler captures of the hot kernels.
 
-Runs one sublayer forward of a workload's shape -- the Attention item or the
-MLP item of one layer, over every budget cell that executes it in the DP
-(E = C - w_item cells x T tokens) -- a few times, with one layer of seeded
-weights and cache.  It holds about 2 GB on the device for the 8B shape, so a
-profiler can replay its kernels quickly.
+``--item attn|mlp`` runs one sublayer forward of a workload's shape -- the
+Attention or the MLP item of one layer, over every budget cell that executes
+it in the DP (E = C - w_item cells x T tokens) -- a few times, with one layer
+of seeded weights and cache.  ``--item solve`` runs whole DP solves of a
+two-layer model of the same shape whose four item weights are set so the
+grid has the workload's full number of cells (every kernel of the loop, the
+select step included, at full width).  About 2-3 GB on the device for the 8B
+shape, so a profiler can replay its kernels quickly.
 
     python -m knapsack_layer_selection_b200.profile_case --workload llama3_8b_8k --item attn
 """
@@ -23,11 +26,13 @@ from knapsack_layer_selection_b200 import workloads as W
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="llama3_8b_8k", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--item", choices=["attn", "mlp"], default="attn")
+    ap.add_argument("--item", choices=["attn", "mlp", "solve"], default="attn")
     ap.add_argument("--repeat", type=int, default=2)
     a = ap.parse_args()
     BUILD.build()
     full = W.WORKLOADS[a.workload]
+    if a.item == "solve":
+        return solve_case(full, a.repeat)
     wl = dataclasses.replace(full, n_layers=1)
     inp = W.make_inputs(wl, device="cuda")
     t = full.latencies()
@@ -49,6 +54,24 @@ def main():
     if st != 0:
         raise SystemExit(f"device status {st}")
     print(f"{a.workload} {a.item}: {E} cells x {wl.T} tokens, {a.repeat} forward(s) ok")
+
+
+def solve_case(full, repeat):
+    wl = dataclasses.replace(full, n_layers=2)
+    inp = W.make_inputs(wl, device="cuda")
+    K = sum(B.quantize_weights(full.latencies(), full.n_bins))
+    w = [K // 4] * 3 + [K - 3 * (K // 4)]          # four items spanning the full grid
+    t = wl.latencies()
+    m = B.model_desc(2, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    s = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, t,
+                 B.params(wl.gamma_max, full.n_bins), w=w, keep_bp=False, keep_tpt=False,
+                 keep_ref=False)
+    for _ in range(repeat):
+        s.solve(inp.x0)
+    torch.cuda.synchronize()
+    s.check_status()
+    print(f"{full.name} solve: 2 layers, {s.C} cells x {wl.T} tokens, {repeat} solve(s) ok")
 
 
 if __name__ == "__main__":
