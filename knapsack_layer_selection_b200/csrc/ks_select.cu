@@ -162,6 +162,14 @@ __device__ __forceinline__ void store_norm4(float* o, float4 v, float sc, const 
                                               v.w * sc * gg.w);
 }
 
+// Four products summed in fp32 (three FMAs), the partial then accumulated in
+// fp64: the rounding of one partial is ~1e-7 of its magnitude, far below the
+// spread of the cosines the select compares, and it keeps fp64 work to one
+// conversion and one add per four elements.
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, a.x * b.x)));
+}
+
 // The DP loop's select step on a state buffer with a leading reference slot:
 // slot 0 holds the full model's state X^(k), slots 1..C the cells 0..C-1.  The
 // batched forward of item k ran on slots 0..E (E = C - w), so exec slot 0 is
@@ -175,7 +183,7 @@ __device__ __forceinline__ void store_norm4(float* o, float4 v, float sc, const 
 // A slot's arithmetic does not depend on its position, so the all-execute cell
 // and the reference slot stay bit-identical.
 template <typename TX, typename TG>
-__global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
+__global__ void __launch_bounds__(kSelectThreads, 2) select_fused_kernel(
     const float* __restrict__ prev, const float* __restrict__ exec,
     const float* __restrict__ target_in, int T, int d, int w, float eps,
     const TG* __restrict__ g_next, float* __restrict__ cur, TX* __restrict__ xh_next,
@@ -204,7 +212,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
   const float* e_base = has_e ? exec + (long long)e_idx * cell : nullptr;
   if (threadIdx.x < 2) hash_sh[threadIdx.x] = 0;
   const float* target = target_in ? target_in : exec;
-  constexpr int U = 4;   // loads issued ahead per lane: keeps enough bytes in flight for HBM
+  constexpr int U = 2;   // loads issued ahead per lane (two CTAs per SM): bytes in flight for HBM
   for (int t = warp; t < T; t += n_warps) {
     const float4* s4 = (const float4*)(s_base + (long long)t * d);
     const float4* r4 = (const float4*)(target + (long long)t * d);
@@ -226,15 +234,15 @@ __global__ void __launch_bounds__(kSelectThreads) select_fused_kernel(
       for (int u = 0; u < U; ++u) {
         if (i0 + 32 * u >= d4) break;
         const float4 a = sv[u];
-        ss += (double)a.x * a.x + (double)a.y * a.y + (double)a.z * a.z + (double)a.w * a.w;
+        ss += (double)dot4(a, a);
         if (!is_ref) {
           const float4 r = rv[u];
-          sr += (double)a.x * r.x + (double)a.y * r.y + (double)a.z * r.z + (double)a.w * r.w;
-          rr += (double)r.x * r.x + (double)r.y * r.y + (double)r.z * r.z + (double)r.w * r.w;
+          sr += (double)dot4(a, r);
+          rr += (double)dot4(r, r);
           if (has_e) {
             const float4 e = ev[u];
-            er += (double)e.x * r.x + (double)e.y * r.y + (double)e.z * r.z + (double)e.w * r.w;
-            ee += (double)e.x * e.x + (double)e.y * e.y + (double)e.z * e.z + (double)e.w * e.w;
+            er += (double)dot4(e, r);
+            ee += (double)dot4(e, e);
           }
         }
       }

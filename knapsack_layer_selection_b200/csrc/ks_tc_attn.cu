@@ -9,27 +9,42 @@
 // compute-bound contraction: O = softmax(Q K^T / sqrt(hd)) V with token t
 // seeing cache positions 0 .. ctx + t.
 //
-// One CTA per (128 query rows, query head); 320 threads:
+// One CTA per (128 query rows, query head); 384 threads in three warpgroups:
 //   warp 0    -- TMA: the Q tile once, then K and V blocks of 128 keys into two
-//                2-slot rings (64-column panels, 128-byte swizzle), K two blocks
-//                ahead of V;
-//   warp 1    -- TMEM owner; one lane issues S_j = Q K_j^T (M=128, N=128) into
-//                one of three S buffers and O += P_j V_j (M=128, N=hd, V read
-//                MN-major straight from the cache layout) into one TMEM
-//                accumulator, in the order S_0, S_1, S_2, PV_0, S_3, PV_1, ...
-//                so two score blocks are in flight while block j's softmax runs;
-//   warps 2-9 -- two threads per query row, each with half of the block's 128
-//                scores and half of the row's O columns (they swap partial row
-//                maxima and, at the end, row sums through shared memory); the
-//                scores of a block go from TMEM to registers once; the running maximum is kept "stale": P is taken
-//                relative to a reference maximum that moves only when the row's
-//                maximum grows by more than 2^8, and only then is the row's O in
-//                TMEM rescaled (after the previous P.V has landed).  exp2 runs
-//                on the MUFU unit for five of every eight scores and as a cubic
-//                on the FMA/integer pipes for the other three.  Only blocks that reach past
-//                position ctx are masked.  P goes to shared memory as bf16 in the
-//                swizzled K-major layout the MMA reads; O is normalised by the
-//                running sum once, at the end.
+//                3-slot rings (64-column panels, 128-byte swizzle);
+//   warp 1    -- TMEM owner; one lane issues S_i = Q K_i^T (M=128, N=128) into
+//                S buffer i%2, as soon as the softmax has copied S_{i-2} out;
+//   warp 2    -- one lane issues O += P_i V_i (M=128, N=hd) with P_i read from
+//                TMEM (P buffer i%2, apart from S) and V read MN-major straight
+//                from the cache layout, as soon as P_i is written.  An MMA
+//                issue returns only as the tensor core takes the work, so with
+//                one issuing thread every barrier wait, fence and commit would
+//                leave the tensor core idle; with two, one thread's waits
+//                overlap the other's MMAs (each commit tracks its own thread's
+//                MMAs, and S and P.V never touch the same TMEM columns);
+//   warp 3    -- idle (it only gives its registers to the softmax);
+//   warps 4-7 and 8-11 -- two softmax groups, one thread per query row (its
+//                TMEM lane) in each: group 0 takes the even blocks, group 1 the
+//                odd ones, so two blocks' softmax run at once and the tensor
+//                core never waits for one.  A group copies its block's 128
+//                scores from TMEM to registers once and frees the S buffer at
+//                once, so S_{i+2} is computed while block i's P is produced.
+//                The running maximum is "stale": block i's reference m_i is
+//                m_{i-1} unless the block's maximum exceeds it by more than 2^8
+//                (in exp2 units), in which case it is the block's maximum and O
+//                in TMEM is rescaled (after PV_{i-1} has landed).  m_i passes
+//                from the group of block i to the other through shared memory,
+//                so both groups' P are taken relative to the same sequence of
+//                references; each group keeps its row sums relative to its last
+//                reference and the two are added, at the end, relative to the
+//                last.  exp2 runs on the MUFU unit for five of every eight
+//                scores and as a cubic on the FMA/integer pipes for the other
+//                three; only blocks that reach past position ctx are masked.
+// Registers: the softmax threads hold a block's 128 scores, so the kernel
+// launches with 168 registers a thread and moves them with setmaxnreg from the
+// first warpgroup (56) to the two softmax warpgroups (224): 128*56 + 256*224 =
+// 384*168, the launch's whole allocation.  The host refuses to launch a build
+// whose register count is not 168, since a larger share could never be met.
 // Every row uses the same block order and the same arithmetic whatever the
 // batch, so a row's output does not depend on the other rows.
 #include <cuda.h>
@@ -43,39 +58,44 @@ using namespace sm100;
 
 namespace {
 
+struct Tail {
+  uint64_t q_full;
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];   // [softmax group = buffer]
+  uint64_t m_ready[2];                                     // [group of the publishing block]
+  uint64_t l_ready;
+  uint64_t drain[2];                                       // [S issuer, PV issuer]
+  uint32_t tmem_base;
+  int abort;
+  float m_pub[2][128];                                     // block references, by block parity
+  float l_pub[128];                                        // the other group's row sums
+};
+
 template <int HD>
 struct Cfg {
-  static constexpr int BM = 128, BN = 128, STAGES = 2;
+  static constexpr int BM = 128, BN = 128, KST = 3;   // rows per tile, keys per block, ring slots
   static constexpr int PANELS = HD / 64;              // 64-wide panels along head_dim
+  static constexpr int Q_PANEL = BM * 128;            // [128 rows][64] bf16
+  static constexpr int Q_TILE = PANELS * Q_PANEL;
   static constexpr int KV_PANEL = BN * 128;           // [128 keys][64] bf16
-  static constexpr int Q_BYTES = BM * HD * 2;
-  static constexpr int K_BYTES = PANELS * KV_PANEL;
-  static constexpr int V_BYTES = PANELS * KV_PANEL;
-  static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int P_PANEL = BM * 128;            // [128 rows][64 keys] bf16
-  static constexpr int P_BYTES = (BN / 64) * P_PANEL;
-  static constexpr int OFF_STAGE = Q_BYTES;
-  static constexpr int OFF_P = Q_BYTES + STAGES * STAGE;
-  static constexpr int OFF_TAIL = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_X = OFF_TAIL + 256;        // [2 blocks][2 halves][128 rows] fp32
-  static constexpr int SMEM = OFF_X + 2 * 2 * BM * 4; // the base is checked to be 1024-aligned
-  static constexpr int THREADS = 320;                 // TMA, MMA, 8 softmax warps
-  static constexpr int S_BUFS = 3;
-  static constexpr int TMEM_S = 0;                    // S buffers: columns [0, 3*BN)
-  static constexpr int TMEM_O = S_BUFS * BN;          // O accumulator: [3*BN, 3*BN + HD)
+  static constexpr int KV_BLOCK = PANELS * KV_PANEL;
+  static constexpr int OFF_K = Q_TILE;
+  static constexpr int OFF_V = OFF_K + KST * KV_BLOCK;
+  static constexpr int OFF_TAIL = OFF_V + KST * KV_BLOCK;
+  static constexpr int USED = OFF_TAIL + (int)((sizeof(Tail) + 255) / 256 * 256);
+  // at least 116 KB, so one CTA holds an SM and its 512 TMEM columns
+  static constexpr int SMEM = USED > 118784 ? USED : 118784;   // base checked 1024-aligned
+  static constexpr int THREADS = 384;                 // TMA, MMA, 2 idle, 2 x 4 softmax warps
+  static constexpr int REGS = 168, REGS_LOW = 56, REGS_HIGH = 224;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH == THREADS * REGS, "register split");
+  static constexpr int TMEM_S = 0;                    // S[b]: columns b * BN (fp32)
+  static constexpr int TMEM_P = 2 * BN;               // P[b]: TMEM_P + b * BN/2 (bf16 pairs)
+  static constexpr int TMEM_O = 3 * BN;               // O: columns TMEM_O .. + HD
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, HD) | (1u << 16);   // B (V) MN-major
-};
-
-struct Tail {
-  uint64_t q_full;
-  uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
-  uint64_t s_full[3], s_free[3], p_full[2], o_done[2];
-  uint64_t pair[2][4];   // per block parity and lane quarter: both halves' values posted
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
+  static_assert(TMEM_O + HD <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(USED <= 232448, "shared memory budget");
 };
 
 struct AttnParams {
@@ -181,8 +201,41 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// Ties 32 registers filled by tcgen05.ld to the point after tcgen05.wait::ld:
+// the compiler sees no dependency between the two instructions, so without
+// this a use of the registers could be scheduled before the wait.
+__device__ __forceinline__ void reg_fence32(float (&v)[32]) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                 "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]),
+                 "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+                 "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]),
+                 "+f"(v[30]), "+f"(v[31]));
+}
+
+// 16 consecutive 32-bit columns (packed bf16 pairs) into this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p_in) {
   using C = Cfg<HD>;
@@ -191,18 +244,16 @@ __global__ void __launch_bounds__(320, 1)
     const long long live = (long long)(*p.dyn_cells) * p.T;
     p.R = (int)(live < p.R ? live : p.R);
   }
-  if ((int)blockIdx.x * C::BM >= p.R) return;   // a row tile past the live rows: nothing to do
+  const int m0 = blockIdx.x * C::BM;
+  if (m0 >= p.R) return;                        // a row tile past the live rows: nothing to do
   extern __shared__ __align__(1024) unsigned char smem[];
-  // the 128-byte-swizzled tiles need a 1024-aligned base; the layout uses all of
-  // shared memory, so there is no room to realign -- refuse instead
+  // the 128-byte-swizzled tiles need a 1024-aligned base; refuse rather than realign
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) raise_status(p.status, KS_ERR_INTERNAL);
     return;
   }
   Tail* tail = reinterpret_cast<Tail*>(smem + C::OFF_TAIL);
-  float* xchg = reinterpret_cast<float*>(smem + C::OFF_X);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * C::BM;
   const int h = blockIdx.y;
   const int g = h / (p.Hq / p.Hkv);
   const int J = p.n_blocks;
@@ -211,21 +262,22 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&tail->q_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::KST; ++s) {
       mbar_init(smem_u32(&tail->k_full[s]), 1);
       mbar_init(smem_u32(&tail->v_full[s]), 1);
       mbar_init(smem_u32(&tail->k_empty[s]), 1);
       mbar_init(smem_u32(&tail->v_empty[s]), 1);
-      mbar_init(smem_u32(&tail->p_full[s]), 256);
-      mbar_init(smem_u32(&tail->o_done[s]), 1);
     }
-    for (int s = 0; s < C::S_BUFS; ++s) {
-      mbar_init(smem_u32(&tail->s_full[s]), 1);
-      mbar_init(smem_u32(&tail->s_free[s]), 256);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tail->s_full[b]), 1);
+      mbar_init(smem_u32(&tail->s_free[b]), 4);         // one arrival per softmax warp
+      mbar_init(smem_u32(&tail->p_full[b]), 4);
+      mbar_init(smem_u32(&tail->pv_done[b]), 1);
+      mbar_init(smem_u32(&tail->m_ready[b]), 4);
     }
-    for (int s = 0; s < 2; ++s)
-      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&tail->pair[s][q]), 64);
-    mbar_init(smem_u32(&tail->drain), 1);
+    mbar_init(smem_u32(&tail->l_ready), 4);
+    mbar_init(smem_u32(&tail->drain[0]), 1);
+    mbar_init(smem_u32(&tail->drain[1]), 1);
     tail->abort = 0;
     fence_barrier_init();
   }
@@ -238,271 +290,288 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
 
-  if (warp == 0) {
+  if (warp < 4) {
+    regs_dec<C::REGS_LOW>();
+    if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const uint32_t qf = smem_u32(&tail->q_full);
-      mbar_arrive_expect_tx(qf, C::Q_BYTES);
+      mbar_arrive_expect_tx(qf, C::Q_TILE);
       for (int pn = 0; pn < C::PANELS; ++pn)
-        tma_load_2d(sbase + pn * (C::BM * 128), &tmQ, h * HD + pn * 64, m0, qf);
-      // K runs two blocks ahead of V, in the order the MMA consumes them:
-      // K_0, K_1, then K_{j+2}, V_j for j = 0, 1, ...
-      auto load_k = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(smem_u32(&tail->k_empty[s]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort,
-                       p.status))
+        tma_load_2d(sbase + pn * C::Q_PANEL, &tmQ, h * HD + pn * 64, m0, qf);
+      // block m of K (V) goes to ring slot m % KST once the MMA of block m - KST is done
+      auto load_kv = [&](const CUtensorMap* tm, int off, uint64_t* full, uint64_t* empty,
+                         int m) -> bool {
+        const int s = m % C::KST;
+        if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(m / C::KST) & 1u) ^ 1u, abort, p.status))
           return false;
-        const uint32_t kst = sbase + C::OFF_STAGE + s * C::STAGE;
-        const uint32_t kf = smem_u32(&tail->k_full[s]);
-        mbar_arrive_expect_tx(kf, C::K_BYTES);
+        const uint32_t dst = sbase + off + s * C::KV_BLOCK;
+        const uint32_t fb = smem_u32(&full[s]);
+        mbar_arrive_expect_tx(fb, C::KV_BLOCK);
         for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_2d(kst + pn * C::KV_PANEL, &tmK, g * HD + pn * 64, j * C::BN, kf);
+          tma_load_2d(dst + pn * C::KV_PANEL, tm, g * HD + pn * 64, m * C::BN, fb);
         return true;
       };
-      auto load_v = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(smem_u32(&tail->v_empty[s]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort,
-                       p.status))
-          return false;
-        const uint32_t vst = sbase + C::OFF_STAGE + s * C::STAGE + C::K_BYTES;
-        const uint32_t vf = smem_u32(&tail->v_full[s]);
-        mbar_arrive_expect_tx(vf, C::V_BYTES);
-        for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_2d(vst + pn * C::KV_PANEL, &tmV, g * HD + pn * 64, j * C::BN, vf);
-        return true;
-      };
+      // in the order the MMAs consume them: K_0, K_1, then K_{j+2}, V_j for j = 0, 1, ...
       int nk = 0, nv = 0;                       // blocks whose K / V loads were issued
       bool ok = true;
-      while (ok && nk < J && nk < 2) ok = load_k(nk++);
+      while (ok && nk < J && nk < 2) {
+        ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk);
+        if (ok) ++nk;
+      }
       while (ok && nv < J) {
         if (nk < J) {
-          if (!(ok = load_k(nk))) break;
+          if (!(ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk))) break;
           ++nk;
         }
-        if (!(ok = load_v(nv))) break;
+        if (!(ok = load_kv(&tmV, C::OFF_V, tail->v_full, tail->v_empty, nv))) break;
         ++nv;
       }
       // drain the copies still in flight before leaving
       mbar_wait_drain(qf, 0, p.status);
-      for (int i = (nk > 2 ? nk - 2 : 0); i < nk; ++i)
-        mbar_wait_drain(smem_u32(&tail->k_full[i & 1]), (uint32_t)(i >> 1) & 1u, p.status);
-      for (int i = (nv > 2 ? nv - 2 : 0); i < nv; ++i)
-        mbar_wait_drain(smem_u32(&tail->v_full[i & 1]), (uint32_t)(i >> 1) & 1u, p.status);
+      for (int i = (nk > C::KST ? nk - C::KST : 0); i < nk; ++i)
+        mbar_wait_drain(smem_u32(&tail->k_full[i % C::KST]), (uint32_t)(i / C::KST) & 1u,
+                        p.status);
+      for (int i = (nv > C::KST ? nv - C::KST : 0); i < nv; ++i)
+        mbar_wait_drain(smem_u32(&tail->v_full[i % C::KST]), (uint32_t)(i / C::KST) & 1u,
+                        p.status);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(smem_u32(&tail->q_full), 0, abort, p.status);
-      tc_fence_after();
-      // S_j = Q K_j^T into S buffer j % 3; released by the softmax once read
-      auto issue_s = [&](int j) -> bool {
-        const int ks = j & 1, sb = j % C::S_BUFS;
-        if (!mbar_wait(smem_u32(&tail->k_full[ks]), (uint32_t)(j >> 1) & 1u, abort, p.status) ||
-            !mbar_wait(smem_u32(&tail->s_free[sb]), ((uint32_t)(j / C::S_BUFS) & 1u) ^ 1u, abort,
-                       p.status))
-          return false;
-        tc_fence_after();
-        const uint32_t kst = sbase + C::OFF_STAGE + ks * C::STAGE;
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- S issuer
+      if (lane == 0) {
+        bool ok = mbar_wait(smem_u32(&tail->q_full), 0, abort, p.status);
+        for (int i = 0; ok && i < J; ++i) {
+          // S_i = Q K_i^T into S buffer i % 2, free once the softmax has copied S_{i-2}
+          const int ks = i % C::KST, b = i & 1;
+          if (i >= 2 && !(ok = mbar_wait(smem_u32(&tail->s_free[b]), ((uint32_t)(i - 2) >> 1) & 1u,
+                                         abort, p.status)))
+            break;
+          if (!(ok = mbar_wait(smem_u32(&tail->k_full[ks]), (uint32_t)(i / C::KST) & 1u, abort,
+                               p.status)))
+            break;
+          tc_fence_after();
+          const uint32_t kst = sbase + C::OFF_K + ks * C::KV_BLOCK;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t a = desc_kmajor_sw128(sbase + (kk / 4) * (C::BM * 128)) + 2 * (kk % 4);
-          const uint64_t b = desc_kmajor_sw128(kst + (kk / 4) * C::KV_PANEL) + 2 * (kk % 4);
-          mma_bf16(tmem + C::TMEM_S + sb * C::BN, a, b, C::IDESC_S, kk > 0);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t a = desc_kmajor_sw128(sbase + (kk / 4) * C::Q_PANEL) + 2 * (kk % 4);
+            const uint64_t bd = desc_kmajor_sw128(kst + (kk / 4) * C::KV_PANEL) + 2 * (kk % 4);
+            mma_bf16(tmem + C::TMEM_S + b * C::BN, a, bd, C::IDESC_S, kk > 0);
+          }
+          mma_commit(smem_u32(&tail->s_full[b]));
+          mma_commit(smem_u32(&tail->k_empty[ks]));
         }
-        mma_commit(smem_u32(&tail->s_full[sb]));
-        mma_commit(smem_u32(&tail->k_empty[ks]));
-        return true;
-      };
-      // O += P_j V_j once the softmax has written P_j
-      auto issue_pv = [&](int i) -> bool {
-        const int s = i & 1;
-        const uint32_t r = (uint32_t)(i >> 1);
-        if (!mbar_wait(smem_u32(&tail->p_full[s]), r & 1u, abort, p.status) ||
-            !mbar_wait(smem_u32(&tail->v_full[s]), r & 1u, abort, p.status))
-          return false;
-        tc_fence_after();
-        const uint32_t pb = sbase + C::OFF_P + s * C::P_BYTES;
-        const uint32_t vst = sbase + C::OFF_STAGE + s * C::STAGE + C::K_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t a = desc_kmajor_sw128(pb + (kk / 4) * C::P_PANEL) + 2 * (kk % 4);
-          // 16 keys = 16 rows of 128 bytes further along K
-          const uint64_t b = desc_mnmajor_sw128(vst + kk * 16 * 128, C::KV_PANEL);
-          mma_bf16(tmem + C::TMEM_O, a, b, C::IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&tail->o_done[s]));
-        mma_commit(smem_u32(&tail->v_empty[s]));
-        return true;
-      };
-      // order: S_0, S_1, then S_{j+2} ahead of PV_j, so two score blocks are in
-      // flight while the softmax of block j runs
-      for (int j = 0; ok && j < J && j < 2; ++j) ok = issue_s(j);
-      for (int j = 0; ok && j < J; ++j) {
-        if (j + 2 < J) ok = issue_s(j + 2);
-        if (ok) ok = issue_pv(j);
+        mma_commit(smem_u32(&tail->drain[0]));
+        mbar_wait_drain(smem_u32(&tail->drain[0]), 0, p.status);
       }
-      mma_commit(smem_u32(&tail->drain));
-      mbar_wait_drain(smem_u32(&tail->drain), 0, p.status);
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- P.V issuer
+      if (lane == 0) {
+        bool ok = true;
+        for (int i = 0; ok && i < J; ++i) {
+          // O += P_i V_i once the softmax has written P_i (into P buffer i % 2)
+          const int vs = i % C::KST, b = i & 1;
+          if (!(ok = mbar_wait(smem_u32(&tail->p_full[b]), ((uint32_t)i >> 1) & 1u, abort,
+                               p.status)))
+            break;
+          if (!(ok = mbar_wait(smem_u32(&tail->v_full[vs]), (uint32_t)(i / C::KST) & 1u, abort,
+                               p.status)))
+            break;
+          tc_fence_after();
+          const uint32_t vst = sbase + C::OFF_V + vs * C::KV_BLOCK;
+          const uint32_t pt = tmem + C::TMEM_P + b * (C::BN / 2);
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            // 16 keys = 8 packed TMEM columns of P, 16 rows of 128 bytes further along V
+            const uint64_t bd = desc_mnmajor_sw128(vst + kk * 16 * 128, C::KV_PANEL);
+            mma_bf16_tmem_a(tmem + C::TMEM_O, pt + kk * 8, bd, C::IDESC_O,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&tail->pv_done[b]));
+          mma_commit(smem_u32(&tail->v_empty[vs]));
+        }
+        mma_commit(smem_u32(&tail->drain[1]));
+        mbar_wait_drain(smem_u32(&tail->drain[1]), 0, p.status);
+      }
     }
   } else {
-    // ------------------------------------------------------------ softmax + output (warps 2-9)
-    // Two warps share each 32-lane quarter of the tile: warp half 0 takes score
-    // and O columns [0, 64) of those rows, half 1 columns [64, 128); they swap
-    // their partial row maxima (and, at the end, row sums) through shared memory.
-    const int q4 = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int r = q4 * 32 + lane;                 // row of the tile = TMEM lane
+    regs_inc<C::REGS_HIGH>();
+    // ------------------------------------------------------------ softmax groups (warps 4-11)
+    const int G = (warp - 4) >> 2;               // group: blocks i with i % 2 == G
+    const int q4 = warp & 3;                     // TMEM lane quarter this warp may access
+    const int r = q4 * 32 + lane;                // row of the tile = TMEM lane
     const int row = m0 + r;
     const bool live = row < p.R;
     const int limit = p.ctx + (live ? row % p.T : 0);   // last visible cache position
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    constexpr int NC = C::BN / 2;                 // score columns per warp
-    constexpr int OC = HD / 2;                    // O columns per warp
+    const uint32_t ts = tmem + lane_off + C::TMEM_S + G * C::BN;
+    const uint32_t tp = tmem + lane_off + C::TMEM_P + G * (C::BN / 2);
+    constexpr int NC = C::BN;                    // scores per row and block
     const float sl2 = p.scale_log2;
-    constexpr float kStale = 8.0f;                // rescale once the max grows by > 2^8
-    float m_ref = -INFINITY;                      // reference maximum (raw score units)
-    float l = 0.f;                                // this half's running sum relative to m_ref
+    constexpr float kStale = 8.0f;               // a new reference once the max grows by > 2^8
+    float m_ref = -INFINITY;                     // reference of this group's last block
+    float l = 0.f;                               // this group's row sum relative to m_ref
     bool ok = true;
-    for (int j = 0; j < J; ++j) {
-      const int s = j & 1;                        // P buffer / O-done barrier of this block
-      const int sb = j % C::S_BUFS;               // S buffer of this block
-      if (!warp_wait(smem_u32(&tail->s_full[sb]), (uint32_t)(j / C::S_BUFS) & 1u, abort,
-                     p.status)) {
+    for (int i = G; i < J; i += 2) {
+      const uint32_t k = (uint32_t)(i >> 1);     // this group's k-th block
+      if (!warp_wait(smem_u32(&tail->s_full[G]), k & 1u, abort, p.status)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t ts = tmem + lane_off + C::TMEM_S + sb * C::BN + half * NC;
-      const int key0 = j * C::BN + half * NC;
-      const bool masked = j * C::BN + C::BN - 1 > p.ctx;   // a key may be past a row's window
       float sc[NC];
 #pragma unroll
       for (int c = 0; c < NC / 32; ++c)
         tmem_ld32(ts + c * 32, *reinterpret_cast<float(*)[32]>(&sc[c * 32]));
       tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < NC / 32; ++c) reg_fence32(*reinterpret_cast<float(*)[32]>(&sc[c * 32]));
       tc_fence_before();
-      mbar_arrive(smem_u32(&tail->s_free[sb]));   // S buffer may be overwritten now
-      if (masked) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tail->s_free[G]));   // S_{i+2} may be computed now
+      if (i * C::BN + C::BN - 1 > p.ctx) {       // a key of this block may be past the window
+        const int key0 = i * C::BN;
 #pragma unroll
         for (int e = 0; e < NC; ++e)
           if (key0 + e > limit) sc[e] = -INFINITY;
       }
-      static_assert(NC % 2 == 0 && NC >= 4, "pairs of scores");
       float mx[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-      for (int e = 4; e < NC; e += 2)             // columns 4 .. NC-1, two at a time
+      for (int e = 4; e < NC; e += 2)            // columns 4 .. NC-1, two at a time
         mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], sc[e], sc[e + 1]);
-      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      // swap half maxima with the partner warp (a bounded wait, like every other)
-      float* xb = xchg + s * (2 * C::BM);
-      xb[half * C::BM + r] = hmax;
-      mbar_arrive(smem_u32(&tail->pair[s][q4]));
-      if (!warp_wait(smem_u32(&tail->pair[s][q4]), (uint32_t)(j >> 1) & 1u, abort, p.status)) {
-        ok = false;
-        break;
-      }
-      const float bmax = fmaxf(hmax, xb[(1 - half) * C::BM + r]);
-      const bool grow = (bmax - m_ref) * sl2 > kStale;   // true on the first block
-      if (__any_sync(0xffffffffu, grow && j > 0)) {
-        // rescale this warp's O columns once the previous P.V has landed in TMEM
-        const int i = j - 1;
-        if (!warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort,
+      const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // the reference of the previous block, from the other group
+      float m_in = -INFINITY;
+      if (i > 0) {
+        const int q = i - 1;
+        if (!warp_wait(smem_u32(&tail->m_ready[1 - G]), ((uint32_t)q >> 1) & 1u, abort,
                        p.status)) {
+          ok = false;
+          break;
+        }
+        m_in = tail->m_pub[1 - G][r];
+      }
+      const bool grow = (bmax - m_in) * sl2 > kStale;   // true on block 0
+      const float m_new = grow ? bmax : m_in;
+      tail->m_pub[G][r] = m_new;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tail->m_ready[G]));
+      if (__any_sync(0xffffffffu, grow && i > 0)) {
+        // O holds the P.V of blocks < i relative to m_in: rescale it once PV_{i-1} has
+        // landed.  The P.V issuer runs behind the S issuer, so the other group's barrier
+        // may still be in the phase of PV_{i-3}, whose parity is the other one: a parity
+        // wait for PV_{i-1} would then pass at once.  Wait for PV_{i-3} first.
+        bool landed = true;
+        for (int q = (i >= 3 ? i - 3 : i - 1); landed && q <= i - 1; q += 2)
+          landed = warp_wait(smem_u32(&tail->pv_done[1 - G]), ((uint32_t)q >> 1) & 1u, abort,
+                             p.status);
+        if (!landed) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float a = grow ? ex2((m_ref - bmax) * sl2) : 1.0f;
+        const float a = grow ? ex2((m_in - m_new) * sl2) : 1.0f;
         float v[32];
 #pragma unroll
-        for (int c = 0; c < OC / 32; ++c) {
-          const uint32_t to = tmem + lane_off + C::TMEM_O + half * OC + c * 32;
+        for (int c = 0; c < HD / 32; ++c) {
+          const uint32_t to = tmem + lane_off + C::TMEM_O + c * 32;
           tmem_ld32(to, v);
           tmem_wait_ld();
+          reg_fence32(v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= a;
           tmem_st32(to, v);
         }
-        tmem_wait_st();
-        l *= a;
       }
-      if (grow) m_ref = bmax;
-      // P_j into shared buffer s: the P.V that last read it (block j-2) must be done
-      if (j >= 2) {
-        const int i = j - 2;
-        if (!warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort,
-                       p.status)) {
-          ok = false;
-          break;
-        }
+      // this group's sum, relative to its previous reference, to the new one
+      if (m_new != m_ref) {
+        l = (m_ref == -INFINITY) ? 0.f : l * ex2((m_ref - m_new) * sl2);
+        m_ref = m_new;
       }
       const uint64_t scale2 = pk2(sl2, sl2);
       const uint64_t moff2 = pk2(-m_ref * sl2, -m_ref * sl2);
       uint64_t sum2[4] = {0, 0, 0, 0};
-      unsigned char* rowp = smem + C::OFF_P + s * C::P_BYTES + half * C::P_PANEL +
-                            (r >> 3) * 1024 + (r & 7) * 128;
+      uint32_t pk[NC / 2];                       // P of the block as bf16 pairs
 #pragma unroll
-      for (int c8 = 0; c8 < NC / 8; ++c8) {       // 8 keys = one 16-byte chunk of the P row
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int k = c8 * 8 + e;
-          float x0, x1, p0, p1;
-          upk2(fma2(pk2(sc[k], sc[k + 1]), scale2, moff2), x0, x1);
-          if ((c8 & 1) ? (e == 2 || e == 6) : (e == 6)) {
-            exp2_cubic2(x0, x1, p0, p1);           // three pairs in eight on the FMA pipe
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          sum2[e >> 1] = add2(sum2[e >> 1], pk2(p0, p1));
-          pk[e >> 1] = pack2(p0, p1);
+      for (int e = 0; e < NC; e += 2) {
+        float x0, x1, p0, p1;
+        upk2(fma2(pk2(sc[e], sc[e + 1]), scale2, moff2), x0, x1);
+        const int pr = (e >> 1) & 7;             // pair index mod 8
+        if (pr == 3 || pr == 5 || pr == 7) {
+          exp2_cubic2(x0, x1, p0, p1);            // three pairs in eight on the FMA pipe
+        } else {
+          p0 = ex2(x0);
+          p1 = ex2(x1);
         }
-        *reinterpret_cast<uint4*>(rowp + ((c8 ^ (r & 7)) * 16)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pk2(p0, p1));
+        pk[e >> 1] = pack2(p0, p1);
       }
+      // P buffer G was last read by PV_{i-2}: wait for it only now, with P in registers
+      if (i >= 2) {
+        const int q = i - 2;
+        if (!warp_wait(smem_u32(&tail->pv_done[G]), ((uint32_t)q >> 1) & 1u, abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < NC / 32; ++c) tmem_st16u(tp + c * 16, &pk[c * 16]);
       float t0, t1, t2, t3, t4, t5, t6, t7;
       upk2(sum2[0], t0, t1);
       upk2(sum2[1], t2, t3);
       upk2(sum2[2], t4, t5);
       upk2(sum2[3], t6, t7);
       l += ((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7));
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // P visible to the MMA
-      tc_fence_before();                          // and any O rescale stores ordered first
-      mbar_arrive(smem_u32(&tail->p_full[s]));
+      tmem_wait_st();                            // P and any O rescale stores complete
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tail->p_full[G]));
     }
-    if (ok && J > 0) {
-      const int i = J - 1;
-      ok = warp_wait(smem_u32(&tail->o_done[i & 1]), (uint32_t)(i >> 1) & 1u, abort, p.status);
+    // the group of the last block holds the final reference; the other group
+    // brings its sum to that reference and hands it over
+    const int last = J - 1, G_last = last & 1;
+    if (ok && G != G_last) {
+      float m_fin = m_ref;
+      if (J > 0) {
+        ok = warp_wait(smem_u32(&tail->m_ready[G_last]), ((uint32_t)last >> 1) & 1u, abort,
+                       p.status);
+        if (ok) m_fin = tail->m_pub[G_last][r];
+      }
+      if (ok) {
+        tail->l_pub[r] = (m_ref == -INFINITY) ? 0.f : l * ex2((m_ref - m_fin) * sl2);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tail->l_ready));
+      }
     }
-    if (ok) {
-      // row sum = both halves' sums (exchanged in the block buffer no block uses now)
-      float* xb = xchg + (J & 1) * (2 * C::BM);
-      xb[half * C::BM + r] = l;
-      mbar_arrive(smem_u32(&tail->pair[J & 1][q4]));
-      ok = warp_wait(smem_u32(&tail->pair[J & 1][q4]), (uint32_t)(J >> 1) & 1u, abort, p.status);
-    }
-    if (ok) {
-      float* xb = xchg + (J & 1) * (2 * C::BM);
-      const float inv = 1.0f / (l + xb[(1 - half) * C::BM + r]);
-      tc_fence_after();
-      uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)p.out +
-                                            ((long long)row * p.Hq + h) * HD + half * OC);
-      float v[32];
+    if (ok && G == G_last) {
+      ok = warp_wait(smem_u32(&tail->l_ready), 0, abort, p.status);
+      if (ok) {
+        l += tail->l_pub[r];
+        ok = warp_wait(smem_u32(&tail->pv_done[G_last]), ((uint32_t)last >> 1) & 1u, abort,
+                       p.status);
+      }
+      if (ok) {
+        const float inv = 1.0f / l;
+        tc_fence_after();
+        uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)p.out +
+                                              ((long long)row * p.Hq + h) * HD);
+        float v[32];
 #pragma unroll
-      for (int c = 0; c < OC / 32; ++c) {
-        tmem_ld32(tmem + lane_off + C::TMEM_O + half * OC + c * 32, v);
-        tmem_wait_ld();
-        if (live) {
+        for (int c = 0; c < HD / 32; ++c) {
+          tmem_ld32(tmem + lane_off + C::TMEM_O + c * 32, v);
+          tmem_wait_ld();
+          reg_fence32(v);
+          if (live) {
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8)
-            dst[c * 4 + q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
-                                         pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
-                                         pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
-                                         pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+            for (int q8 = 0; q8 < 4; ++q8)
+              dst[c * 4 + q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                           pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                           pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                           pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+          }
         }
       }
     }
@@ -517,13 +586,20 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 template <int HD>
-ks_status launch_attn(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
-                      int T, int Hq, int Hkv, int ctx, void* out, int32_t* status,
-                      cudaStream_t st, const int* dyn_cells) {
+ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int T, int Hq, int Hkv,
+                      int ctx, void* out, int32_t* status, cudaStream_t st,
+                      const int* dyn_cells) {
   using C = Cfg<HD>;
   static bool attr = false;
   auto k = attn_kernel<HD>;
   if (!attr) {
+    // the setmaxnreg split assumes exactly C::REGS registers a thread at launch
+    cudaFuncAttributes fa;
+    KS_CUDA_TRY(cudaFuncGetAttributes(&fa, k));
+    if (fa.numRegs != C::REGS)
+      return fail(KS_ERR_INTERNAL, "attention: kernel built with " + std::to_string(fa.numRegs) +
+                                       " registers a thread, the register split needs " +
+                                       std::to_string(C::REGS));
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     attr = true;
   }
@@ -532,7 +608,6 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, long long c
   KS_TRY(make_tmap_2d(&tq, q, R, (long long)Hq * HD, (long long)Hq * HD, 64, C::BM));
   KS_TRY(make_tmap_2d(&tk, kc, n_keys, (long long)Hkv * HD, (long long)Hkv * HD, 64, C::BN));
   KS_TRY(make_tmap_2d(&tv, vc, n_keys, (long long)Hkv * HD, (long long)Hkv * HD, 64, C::BN));
-  (void)cache_rows;
   AttnParams ap;
   ap.out = out;
   ap.status = status;
@@ -545,7 +620,7 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, long long c
   ap.n_blocks = (n_keys + C::BN - 1) / C::BN;
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   ap.dyn_cells = dyn_cells;
-  dim3 grid((R + C::BM - 1) / C::BM, Hq);
+  const dim3 grid((R + C::BM - 1) / C::BM, Hq);
   k<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, ap);
   KS_LAUNCH_CHECK();
   return KS_OK;
@@ -560,9 +635,9 @@ ks_status tc_attention(const void* q, const void* kc, const void* vc, long long 
   if (Hq % Hkv) return fail(KS_ERR_INVALID_ARG, "attention: Hq must be a multiple of Hkv");
   if (cache_rows < (long long)ctx + T) return fail(KS_ERR_INVALID_ARG, "attention: cache too short");
   if (hd == 128)
-    return launch_attn<128>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
+    return launch_attn<128>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
   if (hd == 64)
-    return launch_attn<64>(q, kc, vc, cache_rows, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
+    return launch_attn<64>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
   return fail(KS_ERR_UNSUPPORTED, "attention: head_dim must be 64 or 128");
 }
 
