@@ -13,7 +13,9 @@
 //   warp 0    -- TMA: the Q tile once, then K and V blocks of 128 keys into two
 //                3-slot rings (64-column panels, 128-byte swizzle);
 //   warp 1    -- TMEM owner; one lane issues S_i = Q K_i^T (M=128, N=128) into
-//                S buffer i%2, as soon as the softmax has copied S_{i-2} out;
+//                S buffer i%2, as soon as the softmax has copied S_{i-2} out
+//                (the softmax group that sees S_i complete also frees K_i's
+//                slot, so each S group ends with a single commit);
 //   warp 2    -- one lane issues O += P_i V_i (M=128, N=hd) with P_i read from
 //                TMEM (P buffer i%2, apart from S) and V read MN-major straight
 //                from the cache layout, as soon as P_i is written.  An MMA
@@ -343,6 +345,8 @@ __global__ void __launch_bounds__(384, 1)
       // ---------------------------------------------------------- S issuer
       if (lane == 0) {
         bool ok = mbar_wait(smem_u32(&tail->q_full), 0, abort, p.status);
+        const uint64_t dq0 = desc_kmajor_sw128(sbase);
+        const uint64_t dk0 = desc_kmajor_sw128(sbase + C::OFF_K);
         for (int i = 0; ok && i < J; ++i) {
           // S_i = Q K_i^T into S buffer i % 2, free once the softmax has copied S_{i-2}
           const int ks = i % C::KST, b = i & 1;
@@ -353,15 +357,17 @@ __global__ void __launch_bounds__(384, 1)
                                p.status)))
             break;
           tc_fence_after();
-          const uint32_t kst = sbase + C::OFF_K + ks * C::KV_BLOCK;
+          // descriptors of a tile: the base's plus the byte offset / 16 (shared
+          // addresses stay below 2^18, so the 14-bit start field never carries)
+          const uint64_t dk = dk0 + (uint64_t)((ks * C::KV_BLOCK) >> 4);
+          const uint32_t ds = tmem + C::TMEM_S + b * C::BN;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t a = desc_kmajor_sw128(sbase + (kk / 4) * C::Q_PANEL) + 2 * (kk % 4);
-            const uint64_t bd = desc_kmajor_sw128(kst + (kk / 4) * C::KV_PANEL) + 2 * (kk % 4);
-            mma_bf16(tmem + C::TMEM_S + b * C::BN, a, bd, C::IDESC_S, kk > 0);
-          }
+          for (int kk = 0; kk < HD / 16; ++kk)
+            mma_bf16(ds, dq0 + (uint64_t)((kk / 4) * (C::Q_PANEL >> 4) + 2 * (kk % 4)),
+                     dk + (uint64_t)((kk / 4) * (C::KV_PANEL >> 4) + 2 * (kk % 4)), C::IDESC_S,
+                     kk > 0);
+          // one commit: the softmax group that sees S_i complete frees K slot ks
           mma_commit(smem_u32(&tail->s_full[b]));
-          mma_commit(smem_u32(&tail->k_empty[ks]));
         }
         mma_commit(smem_u32(&tail->drain[0]));
         mbar_wait_drain(smem_u32(&tail->drain[0]), 0, p.status);
@@ -370,6 +376,7 @@ __global__ void __launch_bounds__(384, 1)
       // ---------------------------------------------------------- P.V issuer
       if (lane == 0) {
         bool ok = true;
+        const uint64_t dv0 = desc_mnmajor_sw128(sbase + C::OFF_V, C::KV_PANEL);
         for (int i = 0; ok && i < J; ++i) {
           // O += P_i V_i once the softmax has written P_i (into P buffer i % 2)
           const int vs = i % C::KST, b = i & 1;
@@ -380,15 +387,13 @@ __global__ void __launch_bounds__(384, 1)
                                p.status)))
             break;
           tc_fence_after();
-          const uint32_t vst = sbase + C::OFF_V + vs * C::KV_BLOCK;
+          const uint64_t dv = dv0 + (uint64_t)((vs * C::KV_BLOCK) >> 4);
           const uint32_t pt = tmem + C::TMEM_P + b * (C::BN / 2);
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
+          for (int kk = 0; kk < C::BN / 16; ++kk)
             // 16 keys = 8 packed TMEM columns of P, 16 rows of 128 bytes further along V
-            const uint64_t bd = desc_mnmajor_sw128(vst + kk * 16 * 128, C::KV_PANEL);
-            mma_bf16_tmem_a(tmem + C::TMEM_O, pt + kk * 8, bd, C::IDESC_O,
-                            (i > 0 || kk > 0) ? 1u : 0u);
-          }
+            mma_bf16_tmem_a(tmem + C::TMEM_O, pt + kk * 8, dv + (uint64_t)(kk * ((16 * 128) >> 4)),
+                            C::IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&tail->pv_done[b]));
           mma_commit(smem_u32(&tail->v_empty[vs]));
         }
@@ -420,6 +425,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = false;
         break;
       }
+      if (q4 == 0 && lane == 0) mbar_arrive(smem_u32(&tail->k_empty[i % C::KST]));   // K_i read
       tc_fence_after();
       float sc[NC];
 #pragma unroll
