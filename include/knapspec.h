@@ -212,7 +212,9 @@ KS_API ks_status ks_gemm_bf16(const void* A, const void* B, float* C, const floa
  * with t = r % T and kv head h / (Hq / Hkv).  q, out: device bf16
  * [R][Hq][head_dim]; k_layer, v_layer: device bf16 [cache_rows][Hkv][head_dim]
  * (one layer of the cache); head_dim 64 or 128; cache_rows >= ctx + T.
- * status: device [1] word for a timed-out wait, or NULL.
+ * status: device [1] word for a timed-out wait, or NULL.  KS_ERR_INTERNAL if
+ * the library was built with a register count the kernel's warpgroup register
+ * split does not expect (the launch is refused rather than left to wait).
  */
 KS_API ks_status ks_attention_bf16(const void* q, const void* k_layer, const void* v_layer,
                                    int64_t cache_rows, int32_t R, int32_t T, int32_t Hq,

@@ -179,7 +179,8 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
 //                 (the caller's X^(k+1), or exec slot 0).
 // Every block also writes the next item's normalised operand of the state it
 // stores, x^ = x / sqrt(mean_t(x^2) + eps) * g_next, from the per-token sums of
-// squares the cosine already needs (fp64), so no separate RMSNorm pass runs.
+// squares the cosine already needs (fp32 partials of four products accumulated
+// in fp64), so no separate RMSNorm pass runs.  Two 512-thread CTAs share an SM.
 // A slot's arithmetic does not depend on its position, so the all-execute cell
 // and the reference slot stay bit-identical.
 template <typename TX, typename TG>
