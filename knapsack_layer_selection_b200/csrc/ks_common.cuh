@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 #include "../../include/knapspec.h"
@@ -31,6 +32,20 @@ ks_status fail(ks_status s, const std::string& msg);
 #define KS_LAUNCH_CHECK() KS_CUDA_TRY(cudaGetLastError())
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Runs `set` (a function-attribute setup returning ks_status) once per device
+// for the call site owning `done`: function attributes are per device.  Two
+// threads may both run it the first time, which is harmless.
+template <typename F>
+ks_status once_per_device(std::atomic<unsigned long long>& done, F&& set) {
+  int dev = 0;
+  KS_CUDA_TRY(cudaGetDevice(&dev));
+  const unsigned long long bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load() & bit)) return KS_OK;
+  KS_TRY(set());
+  if (bit) done.fetch_or(bit);
+  return KS_OK;
+}
 
 // ---------------------------------------------------------------- element types
 template <typename T> struct Elem;

@@ -596,9 +596,9 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int 
                       int ctx, void* out, int32_t* status, cudaStream_t st,
                       const int* dyn_cells) {
   using C = Cfg<HD>;
-  static bool attr = false;
+  static std::atomic<unsigned long long> attr{0};
   auto k = attn_kernel<HD>;
-  if (!attr) {
+  KS_TRY(once_per_device(attr, [&]() -> ks_status {
     // the setmaxnreg split assumes exactly C::REGS registers a thread at launch
     cudaFuncAttributes fa;
     KS_CUDA_TRY(cudaFuncGetAttributes(&fa, k));
@@ -607,8 +607,8 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int 
                                        " registers a thread, the register split needs " +
                                        std::to_string(C::REGS));
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-    attr = true;
-  }
+    return KS_OK;
+  }));
   const int n_keys = ctx + T;
   CUtensorMap tq, tk, tv;
   KS_TRY(make_tmap_2d(&tq, q, R, (long long)Hq * HD, (long long)Hq * HD, 64, C::BM));

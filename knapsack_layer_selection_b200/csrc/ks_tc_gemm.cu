@@ -358,12 +358,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 template <int EPI>
 ks_status launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
                  const GemmParams& gp, cudaStream_t st) {
-  static bool attr_set = false;
+  static std::atomic<unsigned long long> attr_set{0};
   auto k = tc_gemm_kernel<EPI>;
-  if (!attr_set) {
+  KS_TRY(once_per_device(attr_set, [&]() -> ks_status {
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    attr_set = true;
-  }
+    return KS_OK;
+  }));
   const int n_tiles = gp.tiles_m * gp.tiles_n;
   const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
   k<<<grid, THREADS, SMEM_BYTES, st>>>(a, b, b2, gp);
