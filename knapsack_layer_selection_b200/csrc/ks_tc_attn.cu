@@ -10,38 +10,41 @@
 // seeing cache positions 0 .. ctx + t.
 //
 // One CTA per (128 query rows, query head); 384 threads in three warpgroups:
-//   warp 0    -- TMA: the Q tile once, then K and V blocks of 128 keys into two
-//                3-slot rings (64-column panels, 128-byte swizzle);
+//   warp 0    -- TMA: the Q tile once, then K blocks of 128 keys into a 3-slot
+//                ring and V blocks into a 2-slot ring (64-column panels,
+//                128-byte swizzle); each V slot ends with a panel of ones;
 //   warp 1    -- TMEM owner; one lane issues S_i = Q K_i^T (M=128, N=128) into
 //                S buffer i%2, as soon as the softmax has copied S_{i-2} out
 //                (the softmax group that sees S_i complete also frees K_i's
 //                slot, so each S group ends with a single commit);
-//   warp 2    -- one lane issues O += P_i V_i (M=128, N=hd) with P_i read from
-//                TMEM (P buffer i%2, apart from S) and V read MN-major straight
-//                from the cache layout, as soon as P_i is written.  An MMA
-//                issue returns only as the tensor core takes the work, so with
-//                one issuing thread every barrier wait, fence and commit would
-//                leave the tensor core idle; with two, one thread's waits
-//                overlap the other's MMAs (each commit tracks its own thread's
-//                MMAs, and S and P.V never touch the same TMEM columns);
+//   warp 2    -- one lane issues [O | l] += P_i [V_i | 1] (M=128, N=hd+16) with
+//                P_i read from TMEM and V read MN-major straight from the cache
+//                layout, as soon as P_i is written: the 16 columns after O
+//                collect P's row sums, so the softmax never adds its
+//                probabilities up.  An MMA issue returns only as the tensor
+//                core takes the work, so with one issuing thread every barrier
+//                wait, fence and commit would leave the tensor core idle; with
+//                two, one thread's waits overlap the other's MMAs (each commit
+//                tracks its own thread's MMAs, and S and P.V never touch the
+//                same TMEM columns);
 //   warp 3    -- idle (it only gives its registers to the softmax);
 //   warps 4-7 and 8-11 -- two softmax groups, one thread per query row (its
 //                TMEM lane) in each: group 0 takes the even blocks, group 1 the
-//                odd ones, so two blocks' softmax run at once and the tensor
-//                core never waits for one.  A group copies its block's 128
-//                scores from TMEM to registers once and frees the S buffer at
-//                once, so S_{i+2} is computed while block i's P is produced.
-//                The running maximum is "stale": block i's reference m_i is
-//                m_{i-1} unless the block's maximum exceeds it by more than 2^8
-//                (in exp2 units), in which case it is the block's maximum and O
-//                in TMEM is rescaled (after PV_{i-1} has landed).  m_i passes
-//                from the group of block i to the other through shared memory,
-//                so both groups' P are taken relative to the same sequence of
-//                references; each group keeps its row sums relative to its last
-//                reference and the two are added, at the end, relative to the
-//                last.  exp2 runs on the MUFU unit for five of every eight
-//                scores and as a cubic on the FMA/integer pipes for the other
-//                three; only blocks that reach past position ctx are masked.
+//                odd ones, so two blocks' softmax run at once.  A group copies
+//                its block's 128 scores from TMEM to registers once and frees
+//                the S buffer at once, so S_{i+2} is computed while block i's P
+//                is produced; P goes to TMEM (one buffer) once PV_{i-1} has read
+//                the previous one.  The running maximum is "stale": block i's
+//                reference m_i is m_{i-1} unless the block's maximum exceeds it
+//                by more than 2^8 (in exp2 units), in which case it is the
+//                block's maximum and O with its row sums is rescaled in TMEM
+//                (after PV_{i-1} has landed).  m_i passes from the group of block
+//                i to the other through shared memory, so both groups' P are taken
+//                relative to the same sequence of references.  exp2 runs on the
+//                MUFU unit for five of every eight scores and as a cubic on the
+//                FMA/integer pipes for the other three; only blocks that reach
+//                past position ctx are masked.  The group of the last block
+//                divides O by its row sum and stores it.
 // Registers: the softmax threads hold a block's 128 scores, so the kernel
 // launches with 168 registers a thread and moves them with setmaxnreg from the
 // first warpgroup (56) to the two softmax warpgroups (224): 128*56 + 256*224 =
@@ -62,28 +65,32 @@ namespace {
 
 struct Tail {
   uint64_t q_full;
-  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];   // [softmax group = buffer]
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];                           // [softmax group = S buffer]
+  uint64_t p_full;                                         // one phase per block
+  uint64_t pv_done[2];                                     // [block parity]: PV_i on pv_done[i % 2]
   uint64_t m_ready[2];                                     // [group of the publishing block]
-  uint64_t l_ready;
   uint64_t drain[2];                                       // [S issuer, PV issuer]
   uint32_t tmem_base;
   int abort;
   float m_pub[2][128];                                     // block references, by block parity
-  float l_pub[128];                                        // the other group's row sums
 };
 
 template <int HD>
 struct Cfg {
-  static constexpr int BM = 128, BN = 128, KST = 3;   // rows per tile, keys per block, ring slots
+  static constexpr int BM = 128, BN = 128, KST = 3, VST = 2;   // rows, keys per block, K / V slots
   static constexpr int PANELS = HD / 64;              // 64-wide panels along head_dim
   static constexpr int Q_PANEL = BM * 128;            // [128 rows][64] bf16
   static constexpr int Q_TILE = PANELS * Q_PANEL;
   static constexpr int KV_PANEL = BN * 128;           // [128 keys][64] bf16
   static constexpr int KV_BLOCK = PANELS * KV_PANEL;
+  // a V slot holds the block's PANELS panels of V and one panel of ones after
+  // them: the P.V MMA reads N = HD + 16 columns, the last 16 giving P's row sums
+  static constexpr int V_SLOT = (PANELS + 1) * KV_PANEL;
+  static constexpr int N_O = HD + 16;
   static constexpr int OFF_K = Q_TILE;
   static constexpr int OFF_V = OFF_K + KST * KV_BLOCK;
-  static constexpr int OFF_TAIL = OFF_V + KST * KV_BLOCK;
+  static constexpr int OFF_TAIL = OFF_V + VST * V_SLOT;
   static constexpr int USED = OFF_TAIL + (int)((sizeof(Tail) + 255) / 256 * 256);
   // at least 116 KB, so one CTA holds an SM and its 512 TMEM columns
   static constexpr int SMEM = USED > 118784 ? USED : 118784;   // base checked 1024-aligned
@@ -91,12 +98,12 @@ struct Cfg {
   static constexpr int REGS = 168, REGS_LOW = 56, REGS_HIGH = 224;
   static_assert(128 * REGS_LOW + 256 * REGS_HIGH == THREADS * REGS, "register split");
   static constexpr int TMEM_S = 0;                    // S[b]: columns b * BN (fp32)
-  static constexpr int TMEM_P = 2 * BN;               // P[b]: TMEM_P + b * BN/2 (bf16 pairs)
-  static constexpr int TMEM_O = 3 * BN;               // O: columns TMEM_O .. + HD
+  static constexpr int TMEM_P = 2 * BN;               // P: TMEM_P .. + BN/2 (bf16 pairs)
+  static constexpr int TMEM_O = 2 * BN + BN / 2;      // O: HD columns, then 16 of row sums
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN);
-  static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, HD) | (1u << 16);   // B (V) MN-major
-  static_assert(TMEM_O + HD <= (int)TMEM_COLS, "TMEM budget");
+  static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, N_O) | (1u << 16);   // B (V) MN-major
+  static_assert(TMEM_O + N_O <= (int)TMEM_COLS, "TMEM budget");
   static_assert(USED <= 232448, "shared memory budget");
 };
 
@@ -266,18 +273,20 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(&tail->q_full), 1);
     for (int s = 0; s < C::KST; ++s) {
       mbar_init(smem_u32(&tail->k_full[s]), 1);
-      mbar_init(smem_u32(&tail->v_full[s]), 1);
       mbar_init(smem_u32(&tail->k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
+      mbar_init(smem_u32(&tail->v_full[s]), 1);
       mbar_init(smem_u32(&tail->v_empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tail->s_full[b]), 1);
       mbar_init(smem_u32(&tail->s_free[b]), 4);         // one arrival per softmax warp
-      mbar_init(smem_u32(&tail->p_full[b]), 4);
-      mbar_init(smem_u32(&tail->pv_done[b]), 1);
       mbar_init(smem_u32(&tail->m_ready[b]), 4);
     }
-    mbar_init(smem_u32(&tail->l_ready), 4);
+    mbar_init(smem_u32(&tail->p_full), 4);
+    mbar_init(smem_u32(&tail->pv_done[0]), 1);
+    mbar_init(smem_u32(&tail->pv_done[1]), 1);
     mbar_init(smem_u32(&tail->drain[0]), 1);
     mbar_init(smem_u32(&tail->drain[1]), 1);
     tail->abort = 0;
@@ -287,6 +296,14 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(&tail->tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // the ones panel of each V slot (every element 1.0, so its swizzle is moot);
+  // the TMA only ever writes the V panels before it
+  for (int s = 0; s < C::VST; ++s) {
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::OFF_V + s * C::V_SLOT + C::PANELS * C::KV_PANEL);
+    for (int e = threadIdx.x; e < C::KV_PANEL / 16; e += blockDim.x)
+      ones[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -306,11 +323,11 @@ __global__ void __launch_bounds__(384, 1)
         tma_load_2d(sbase + pn * C::Q_PANEL, &tmQ, h * HD + pn * 64, m0, qf);
       // block m of K (V) goes to ring slot m % KST once the MMA of block m - KST is done
       auto load_kv = [&](const CUtensorMap* tm, int off, uint64_t* full, uint64_t* empty,
-                         int m) -> bool {
-        const int s = m % C::KST;
-        if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(m / C::KST) & 1u) ^ 1u, abort, p.status))
+                         int m, int nst, int slot_bytes) -> bool {
+        const int s = m % nst;
+        if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(m / nst) & 1u) ^ 1u, abort, p.status))
           return false;
-        const uint32_t dst = sbase + off + s * C::KV_BLOCK;
+        const uint32_t dst = sbase + off + s * slot_bytes;
         const uint32_t fb = smem_u32(&full[s]);
         mbar_arrive_expect_tx(fb, C::KV_BLOCK);
         for (int pn = 0; pn < C::PANELS; ++pn)
@@ -321,15 +338,15 @@ __global__ void __launch_bounds__(384, 1)
       int nk = 0, nv = 0;                       // blocks whose K / V loads were issued
       bool ok = true;
       while (ok && nk < J && nk < 2) {
-        ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk);
+        ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST, C::KV_BLOCK);
         if (ok) ++nk;
       }
       while (ok && nv < J) {
         if (nk < J) {
-          if (!(ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk))) break;
+          if (!(ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST, C::KV_BLOCK))) break;
           ++nk;
         }
-        if (!(ok = load_kv(&tmV, C::OFF_V, tail->v_full, tail->v_empty, nv))) break;
+        if (!(ok = load_kv(&tmV, C::OFF_V, tail->v_full, tail->v_empty, nv, C::VST, C::V_SLOT))) break;
         ++nv;
       }
       // drain the copies still in flight before leaving
@@ -337,8 +354,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int i = (nk > C::KST ? nk - C::KST : 0); i < nk; ++i)
         mbar_wait_drain(smem_u32(&tail->k_full[i % C::KST]), (uint32_t)(i / C::KST) & 1u,
                         p.status);
-      for (int i = (nv > C::KST ? nv - C::KST : 0); i < nv; ++i)
-        mbar_wait_drain(smem_u32(&tail->v_full[i % C::KST]), (uint32_t)(i / C::KST) & 1u,
+      for (int i = (nv > C::VST ? nv - C::VST : 0); i < nv; ++i)
+        mbar_wait_drain(smem_u32(&tail->v_full[i % C::VST]), (uint32_t)(i / C::VST) & 1u,
                         p.status);
     }
     } else if (warp == 1) {
@@ -378,23 +395,22 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         const uint64_t dv0 = desc_mnmajor_sw128(sbase + C::OFF_V, C::KV_PANEL);
         for (int i = 0; ok && i < J; ++i) {
-          // O += P_i V_i once the softmax has written P_i (into P buffer i % 2)
-          const int vs = i % C::KST, b = i & 1;
-          if (!(ok = mbar_wait(smem_u32(&tail->p_full[b]), ((uint32_t)i >> 1) & 1u, abort,
-                               p.status)))
+          // [O | row sums] += P_i [V_i | ones] once the softmax has written P_i
+          const int vs = i % C::VST;
+          if (!(ok = mbar_wait(smem_u32(&tail->p_full), (uint32_t)i & 1u, abort, p.status)))
             break;
-          if (!(ok = mbar_wait(smem_u32(&tail->v_full[vs]), (uint32_t)(i / C::KST) & 1u, abort,
+          if (!(ok = mbar_wait(smem_u32(&tail->v_full[vs]), (uint32_t)(i / C::VST) & 1u, abort,
                                p.status)))
             break;
           tc_fence_after();
-          const uint64_t dv = dv0 + (uint64_t)((vs * C::KV_BLOCK) >> 4);
-          const uint32_t pt = tmem + C::TMEM_P + b * (C::BN / 2);
+          const uint64_t dv = dv0 + (uint64_t)((vs * C::V_SLOT) >> 4);
+          const uint32_t pt = tmem + C::TMEM_P;
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
             // 16 keys = 8 packed TMEM columns of P, 16 rows of 128 bytes further along V
             mma_bf16_tmem_a(tmem + C::TMEM_O, pt + kk * 8, dv + (uint64_t)(kk * ((16 * 128) >> 4)),
                             C::IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&tail->pv_done[b]));
+          mma_commit(smem_u32(&tail->pv_done[i & 1]));
           mma_commit(smem_u32(&tail->v_empty[vs]));
         }
         mma_commit(smem_u32(&tail->drain[1]));
@@ -412,13 +428,22 @@ __global__ void __launch_bounds__(384, 1)
     const int limit = p.ctx + (live ? row % p.T : 0);   // last visible cache position
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t ts = tmem + lane_off + C::TMEM_S + G * C::BN;
-    const uint32_t tp = tmem + lane_off + C::TMEM_P + G * (C::BN / 2);
+    const uint32_t tp = tmem + lane_off + C::TMEM_P;
     constexpr int NC = C::BN;                    // scores per row and block
     const float sl2 = p.scale_log2;
     constexpr float kStale = 8.0f;               // a new reference once the max grows by > 2^8
-    float m_ref = -INFINITY;                     // reference of this group's last block
-    float l = 0.f;                               // this group's row sum relative to m_ref
     bool ok = true;
+    // waits until PV_q has completed.  PV_q commits to pv_done[q % 2], whose phases
+    // are PV_{q-2}, PV_q, PV_{q+2}...; at every wait below PV_{q-2} has completed
+    // (this group waited for it, or for a later P.V, whose commit covers it) and
+    // PV_{q+2} cannot have (it needs a P this group has not yet written), so a
+    // parity wait sees the right phase
+    auto wait_pv = [&](int q) -> bool {
+      if (!warp_wait(smem_u32(&tail->pv_done[q & 1]), ((uint32_t)q >> 1) & 1u, abort, p.status))
+        return false;
+      tc_fence_after();
+      return true;
+    };
     for (int i = G; i < J; i += 2) {
       const uint32_t k = (uint32_t)(i >> 1);     // this group's k-th block
       if (!warp_wait(smem_u32(&tail->s_full[G]), k & 1u, abort, p.status)) {
@@ -465,19 +490,12 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tail->m_ready[G]));
       if (__any_sync(0xffffffffu, grow && i > 0)) {
-        // O holds the P.V of blocks < i relative to m_in: rescale it once PV_{i-1} has
-        // landed.  The P.V issuer runs behind the S issuer, so the other group's barrier
-        // may still be in the phase of PV_{i-3}, whose parity is the other one: a parity
-        // wait for PV_{i-1} would then pass at once.  Wait for PV_{i-3} first.
-        bool landed = true;
-        for (int q = (i >= 3 ? i - 3 : i - 1); landed && q <= i - 1; q += 2)
-          landed = warp_wait(smem_u32(&tail->pv_done[1 - G]), ((uint32_t)q >> 1) & 1u, abort,
-                             p.status);
-        if (!landed) {
+        // O and its row sums hold the P.V of blocks < i relative to m_in: rescale them
+        // once PV_{i-1} has landed
+        if (!wait_pv(i - 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const float a = grow ? ex2((m_in - m_new) * sl2) : 1.0f;
         float v[32];
 #pragma unroll
@@ -490,15 +508,19 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < 32; ++e) v[e] *= a;
           tmem_st32(to, v);
         }
-      }
-      // this group's sum, relative to its previous reference, to the new one
-      if (m_new != m_ref) {
-        l = (m_ref == -INFINITY) ? 0.f : l * ex2((m_ref - m_new) * sl2);
-        m_ref = m_new;
+        {
+          const uint32_t to = tmem + lane_off + C::TMEM_O + HD;   // the 16 row-sum columns
+          tmem_wait_st();                        // the stores above land before this reload
+          tmem_ld32(to - 16, v);                 // 32 columns ending at the sums: HD-16 .. HD+15
+          tmem_wait_ld();
+          reg_fence32(v);
+#pragma unroll
+          for (int e = 16; e < 32; ++e) v[e] *= a;   // the first 16 were rescaled above
+          tmem_st32(to - 16, v);
+        }
       }
       const uint64_t scale2 = pk2(sl2, sl2);
-      const uint64_t moff2 = pk2(-m_ref * sl2, -m_ref * sl2);
-      uint64_t sum2[4] = {0, 0, 0, 0};
+      const uint64_t moff2 = pk2(-m_new * sl2, -m_new * sl2);
       uint32_t pk[NC / 2];                       // P of the block as bf16 pairs
 #pragma unroll
       for (int e = 0; e < NC; e += 2) {
@@ -511,73 +533,42 @@ __global__ void __launch_bounds__(384, 1)
           p0 = ex2(x0);
           p1 = ex2(x1);
         }
-        sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pk2(p0, p1));
         pk[e >> 1] = pack2(p0, p1);
       }
-      // P buffer G was last read by PV_{i-2}: wait for it only now, with P in registers
-      if (i >= 2) {
-        const int q = i - 2;
-        if (!warp_wait(smem_u32(&tail->pv_done[G]), ((uint32_t)q >> 1) & 1u, abort, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      // the P buffer was last read by PV_{i-1}: wait for it only now, with P in registers
+      if (i >= 1 && !wait_pv(i - 1)) {
+        ok = false;
+        break;
       }
 #pragma unroll
       for (int c = 0; c < NC / 32; ++c) tmem_st16u(tp + c * 16, &pk[c * 16]);
-      float t0, t1, t2, t3, t4, t5, t6, t7;
-      upk2(sum2[0], t0, t1);
-      upk2(sum2[1], t2, t3);
-      upk2(sum2[2], t4, t5);
-      upk2(sum2[3], t6, t7);
-      l += ((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7));
       tmem_wait_st();                            // P and any O rescale stores complete
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tail->p_full[G]));
+      if (lane == 0) mbar_arrive(smem_u32(&tail->p_full));
     }
-    // the group of the last block holds the final reference; the other group
-    // brings its sum to that reference and hands it over
-    const int last = J - 1, G_last = last & 1;
-    if (ok && G != G_last) {
-      float m_fin = m_ref;
-      if (J > 0) {
-        ok = warp_wait(smem_u32(&tail->m_ready[G_last]), ((uint32_t)last >> 1) & 1u, abort,
-                       p.status);
-        if (ok) m_fin = tail->m_pub[G_last][r];
-      }
-      if (ok) {
-        tail->l_pub[r] = (m_ref == -INFINITY) ? 0.f : l * ex2((m_ref - m_fin) * sl2);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tail->l_ready));
-      }
-    }
-    if (ok && G == G_last) {
-      ok = warp_wait(smem_u32(&tail->l_ready), 0, abort, p.status);
-      if (ok) {
-        l += tail->l_pub[r];
-        ok = warp_wait(smem_u32(&tail->pv_done[G_last]), ((uint32_t)last >> 1) & 1u, abort,
-                       p.status);
-      }
-      if (ok) {
-        const float inv = 1.0f / l;
-        tc_fence_after();
-        uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)p.out +
-                                              ((long long)row * p.Hq + h) * HD);
-        float v[32];
+    // the group of the last block writes the output: O over its row sum
+    const int last = J - 1;
+    if (ok && G == (last & 1) && wait_pv(last)) {
+      float v[32];
+      tmem_ld32(tmem + lane_off + C::TMEM_O + HD - 16, v);   // HD-16 .. HD+15: the sum at 16
+      tmem_wait_ld();
+      reg_fence32(v);
+      const float inv = 1.0f / v[16];
+      uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)p.out +
+                                            ((long long)row * p.Hq + h) * HD);
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          tmem_ld32(tmem + lane_off + C::TMEM_O + c * 32, v);
-          tmem_wait_ld();
-          reg_fence32(v);
-          if (live) {
+      for (int c = 0; c < HD / 32; ++c) {
+        tmem_ld32(tmem + lane_off + C::TMEM_O + c * 32, v);
+        tmem_wait_ld();
+        reg_fence32(v);
+        if (live) {
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-              dst[c * 4 + q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
-                                           pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
-                                           pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
-                                           pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
-          }
+          for (int q8 = 0; q8 < 4; ++q8)
+            dst[c * 4 + q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                         pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                         pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                         pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
         }
       }
     }
