@@ -15,6 +15,10 @@
  * (Eq. 4, Eq. 5).
  *
  * Conventions shared by every call:
+ *  - The comments below label the steps of the solve a0 .. a6: a0 item weights
+ *    and the budget grid, a1 the full model's reference states, a2 / a3 the
+ *    Attention / MLP item on a batch of states, a4 the select with its
+ *    backpointer, a5 the set reconstruction, a6 the TPT grid search.
  *  - Items are numbered k = 0 .. 2L-1: item 2l is the Attention sublayer of
  *    layer l, item 2l+1 its MLP sublayer.  X^(0) is the T evaluation tokens'
  *    input state, X^(k+1) = item_k(X^(k)).
@@ -313,7 +317,7 @@ KS_API ks_status ks_tpt_argmax(const float* values, const double* t_draft, int32
                         ks_stream_t stream);
 
 /*
- * a0-a6 -- the whole DP on one GPU (the spec call).
+ * a0-a6 -- the whole DP on one GPU (the library's main entry).
  * layers: HOST array [n_layers] of device weight pointers; cache: the full
  * model's KV cache; x0: device [T][d] fp32; ref: device [n_items+1][T][d] fp32
  * reference states to compare against, or NULL to use the ones the solve
