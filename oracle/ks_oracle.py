@@ -22,6 +22,11 @@ which paraphrases the paper's equations:
 * selection -- TPT(S, gamma) = ((1 - a^(gamma+1)) / (1 - a)) / (gamma t_Draft(S)
   + t_Target) maximised over the candidate pool and gamma <= D (Eq. 4, Eq. 5).
 
+Section labels below name the steps of the solve: a0 item weights and the
+budget grid, a1 reference states, a2 / a3 the Attention / MLP sublayer on a
+batch of states, a4 the select with its backpointer, a5 the reconstruction,
+a6 the TPT grid search.
+
 Readings where the page is silent or ambiguous (each is one switch or one line
 below and is listed with its reason in the design notes):
 
