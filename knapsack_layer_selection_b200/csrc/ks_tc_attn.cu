@@ -41,10 +41,11 @@
 //                (after PV_{i-1} has landed).  m_i passes from the group of block
 //                i to the other through shared memory, so both groups' P are taken
 //                relative to the same sequence of references.  exp2 runs on the
-//                MUFU unit for five of every eight scores and as a cubic on the
-//                FMA/integer pipes for the other three; only blocks that reach
-//                past position ctx are masked.  The group of the last block
-//                divides O by its row sum and stores it.
+//                MUFU unit (with the row sums on the tensor core, the softmax is
+//                bound by its instruction count, not by MUFU: moving part of the
+//                exponentials to an FMA-pipe polynomial was measured slower); only
+//                blocks that reach past position ctx are masked.  The group of
+//                the last block divides O by its row sum and stores it.
 // Registers: the softmax threads hold a block's 128 scores, so the kernel
 // launches with 168 registers a thread and moves them with setmaxnreg from the
 // first warpgroup (56) to the two softmax warpgroups (224): 128*56 + 256*224 =
@@ -135,36 +136,10 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for a pair of arguments as 2^n * q(x - n) with n = round(x): adding
-// 1.5 * 2^23 leaves n in the low mantissa bits (and, shifted by 23, exactly the
-// exponent increment), so no conversion instruction is needed; q is a cubic
-// fitted to 2^f on [-1/2, 1/2] for minimal relative error (7.5e-5, far below
-// the bf16 rounding of P).  Every step runs on the FMA or integer pipes, two
-// lanes per f32x2 instruction, which takes load off the MUFU unit.
-__device__ __forceinline__ void exp2_cubic2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t x = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));   // results stay normal
-  const uint64_t t = add2(x, pk2(12582912.0f, 12582912.0f));
-  const uint64_t n = add2(t, pk2(-12582912.0f, -12582912.0f));     // round(x) as a float
-  const uint64_t f = fma2(n, pk2(-1.0f, -1.0f), x);                // x - round(x)
-  uint64_t q = fma2(pk2(0.055171434f, 0.055171434f), f, pk2(0.24261081f, 0.24261081f));
-  q = fma2(q, f, pk2(0.69326097f, 0.69326097f));
-  q = fma2(q, f, pk2(0.99992812f, 0.99992812f));
-  float q0, q1, t0, t1;
-  upk2(q, q0, q1);
-  upk2(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // 32 consecutive fp32 columns into this thread's TMEM lane (32x32b shape, x32).
@@ -526,13 +501,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int e = 0; e < NC; e += 2) {
         float x0, x1, p0, p1;
         upk2(fma2(pk2(sc[e], sc[e + 1]), scale2, moff2), x0, x1);
-        const int pr = (e >> 1) & 7;             // pair index mod 8
-        if (pr == 3 || pr == 5 || pr == 7) {
-          exp2_cubic2(x0, x1, p0, p1);            // three pairs in eight on the FMA pipe
-        } else {
-          p0 = ex2(x0);
-          p1 = ex2(x1);
-        }
+        p0 = ex2(x0);
+        p1 = ex2(x1);
         pk[e >> 1] = pack2(p0, p1);
       }
       // the P buffer was last read by PV_{i-1}: wait for it only now, with P in registers
