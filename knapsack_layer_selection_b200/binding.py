@@ -2,8 +2,11 @@
 
 Every function here only marshals arguments: it checks tensor devices, dtypes
 and shapes, turns them into pointers and calls the C ABI on the current torch
-CUDA stream.  All arithmetic of the DP runs in the library's CUDA kernels.  If
-the library has not been built the first call raises; there is no fallback.
+CUDA stream.  The C ABI takes bare pointers and cannot see a buffer's size, so
+every shape the header fixes is checked here against the sizes passed beside
+it: a wrongly sized tensor raises instead of reaching a kernel.  All arithmetic
+of the DP runs in the library's CUDA kernels.  If the library has not been
+built the first call raises; there is no fallback.
 """
 from __future__ import annotations
 
@@ -130,11 +133,27 @@ def _dev(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
         return None
     if not t.is_cuda:
         raise KnapSpecError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise KnapSpecError(f"{name} is on {t.device}, but calls run on the current device "
+                            f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise KnapSpecError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise KnapSpecError(f"{name} must be {dtype}, got {t.dtype}")
     return t.data_ptr()
+
+
+def _shape(t: Optional[torch.Tensor], shape: Sequence[int], name: str) -> None:
+    """Raise unless t is None or has exactly this shape."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise KnapSpecError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _rows(t: torch.Tensor, n: int, row: Sequence[int], name: str) -> None:
+    """Raise unless t is [m][*row] with m >= n (a buffer of at least n rows)."""
+    if t.dim() != 1 + len(row) or tuple(t.shape[1:]) != tuple(row) or t.shape[0] < n:
+        raise KnapSpecError(f"{name} must have shape (>= {n}, {', '.join(map(str, row))}), "
+                            f"got {tuple(t.shape)}")
 
 
 def _stream() -> int:
@@ -152,7 +171,22 @@ def model_desc(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, ffn, rms_eps,
                      rope_base, KS_F32 if wdtype == "f32" else KS_BF16)
 
 
-def layer_array(layers: Sequence[Dict[str, torch.Tensor]], wdtype: torch.dtype):
+def _layer_shapes(m: ModelDesc) -> Dict[str, tuple]:
+    d, qd, F = m.d_model, m.n_q_heads * m.head_dim, m.ffn
+    return {"attn_norm": (d,), "wq": (qd, d), "wo": (d, qd), "mlp_norm": (d,),
+            "w_gate": (F, d), "w_up": (F, d), "w_down": (d, F)}
+
+
+def layer_array(layers: Sequence[Dict[str, torch.Tensor]], wdtype: torch.dtype,
+                model: Optional[ModelDesc] = None):
+    """Host array of the layers' device weight pointers; with a model, the
+    layer count and every weight's shape are checked against it."""
+    if model is not None and len(layers) != model.n_layers:
+        raise KnapSpecError(f"model has {model.n_layers} layers, got {len(layers)}")
+    if model is not None:
+        for i, L in enumerate(layers):
+            for name, shape in _layer_shapes(model).items():
+                _shape(L[name], shape, f"layers[{i}].{name}")
     arr = (LayerWeights * len(layers))()
     for i, L in enumerate(layers):
         for name in ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down"):
@@ -160,10 +194,20 @@ def layer_array(layers: Sequence[Dict[str, torch.Tensor]], wdtype: torch.dtype):
     return arr
 
 
-def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int) -> CacheDesc:
+def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int,
+               model: Optional[ModelDesc] = None) -> CacheDesc:
+    """The KV cache [L][rows][Hkv][hd] of K and V; with a model, L >= n_layers,
+    Hkv, hd and the dtype are checked against it."""
     if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
         raise KnapSpecError("k_cache / v_cache must both be [L][rows][Hkv][hd]")
-    return CacheDesc(_dev(k_cache, name="k_cache"), _dev(v_cache, name="v_cache"),
+    dt = None
+    if model is not None:
+        L, _, Hkv, hd = k_cache.shape
+        if L < model.n_layers or Hkv != model.n_kv_heads or hd != model.head_dim:
+            raise KnapSpecError(f"k_cache / v_cache must be [>= {model.n_layers}][rows]"
+                                f"[{model.n_kv_heads}][{model.head_dim}], got {tuple(k_cache.shape)}")
+        dt = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
+    return CacheDesc(_dev(k_cache, dt, "k_cache"), _dev(v_cache, dt, "v_cache"),
                      k_cache.shape[1], ctx)
 
 
@@ -200,14 +244,23 @@ def sublayer_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, item: i
                      states_in: torch.Tensor, states_out: torch.Tensor,
                      ws: torch.Tensor) -> None:
     E = states_in.shape[0] if states_in.dim() == 3 else 1
+    _shape(states_in, (E, T, model.d_model) if states_in.dim() == 3 else (T, model.d_model),
+           "states_in")
+    _shape(states_out, tuple(states_in.shape), "states_out")
     _check(load().ks_sublayer_forward(ctypes.byref(model), layers, ctypes.byref(cache), T, item,
                                       _dev(states_in, torch.float32, "states_in"), E,
                                       _dev(states_out, torch.float32, "states_out"),
                                       _dev(ws, name="workspace"), ws.numel(), _stream()))
 
 
+def _ref_shapes(model: ModelDesc, T: int, x0: torch.Tensor, ref_out: torch.Tensor) -> None:
+    _shape(x0, (T, model.d_model), "x0")
+    _shape(ref_out, (2 * model.n_layers + 1, T, model.d_model), "ref_out")
+
+
 def reference_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, x0: torch.Tensor,
                       ref_out: torch.Tensor, ws: torch.Tensor) -> None:
+    _ref_shapes(model, T, x0, ref_out)
     _check(load().ks_reference_forward(ctypes.byref(model), layers, ctypes.byref(cache), T,
                                        _dev(x0, torch.float32, "x0"),
                                        _dev(ref_out, torch.float32, "ref_out"),
@@ -217,6 +270,7 @@ def reference_forward(model: ModelDesc, layers, cache: CacheDesc, T: int, x0: to
 def reference_forward_noalloc(model: ModelDesc, layers, cache: CacheDesc, T: int,
                               x0: torch.Tensor, ref_out: torch.Tensor) -> None:
     """ks_reference_forward using the library's fixed scratch array (no workspace)."""
+    _ref_shapes(model, T, x0, ref_out)
     _check(load().ks_reference_forward_noalloc(ctypes.byref(model), layers, ctypes.byref(cache),
                                                T, _dev(x0, torch.float32, "x0"),
                                                _dev(ref_out, torch.float32, "ref_out"),
@@ -236,6 +290,11 @@ def gemm_bf16(A: torch.Tensor, Bw: torch.Tensor, C: torch.Tensor,
     """C = A . Bw^T (+ resid) on the tensor cores (A [M][K], Bw [N][K] bf16; C fp32)."""
     M, K = A.shape
     N = Bw.shape[0]
+    _shape(Bw, (N, K), "B")
+    _shape(C, (M, N), "C")
+    _shape(resid, (M, N), "resid")
+    if status is not None and status.numel() < 1:
+        raise KnapSpecError("status must hold one int32")
     _check(load().ks_gemm_bf16(_dev(A, torch.bfloat16, "A"), _dev(Bw, torch.bfloat16, "B"),
                                _dev(C, torch.float32, "C"), _dev(resid, torch.float32, "resid"),
                                M, N, K, _dev(status, torch.int32, "status"), _stream()))
@@ -246,6 +305,11 @@ def attention_bf16(q: torch.Tensor, k_layer: torch.Tensor, v_layer: torch.Tensor
     """Tensor-core causal GQA attention: q/out [R][Hq][hd], k/v [rows][Hkv][hd] (bf16)."""
     R, Hq, hd = q.shape
     rows, Hkv, _ = k_layer.shape
+    _shape(k_layer, (rows, Hkv, hd), "k_layer")
+    _shape(v_layer, (rows, Hkv, hd), "v_layer")
+    _shape(out, (R, Hq, hd), "out")
+    if status is not None and status.numel() < 1:
+        raise KnapSpecError("status must hold one int32")
     _check(load().ks_attention_bf16(_dev(q, torch.bfloat16, "q"), _dev(k_layer, torch.bfloat16, "k"),
                                     _dev(v_layer, torch.bfloat16, "v"), rows, R, T, Hq, Hkv, hd,
                                     ctx, _dev(out, torch.bfloat16, "out"),
@@ -261,6 +325,12 @@ def check_bounded_wait(limit_us: int, status: torch.Tensor,
 
 def select_step(prev, exec_, target, w: int, cur, val, bp, cos_skip=None, cos_exec=None) -> None:
     C, T, d = prev.shape
+    if C > w:
+        _rows(exec_, C - w, (T, d), "exec")
+    _shape(target, (T, d), "target")
+    _shape(cur, (C, T, d), "cur")
+    for t, name in ((val, "val"), (bp, "bp"), (cos_skip, "cos_skip"), (cos_exec, "cos_exec")):
+        _shape(t, (C,), name)
     _check(load().ks_select_step(_dev(prev, torch.float32, "prev"),
                                  _dev(exec_, torch.float32, "exec"),
                                  _dev(target, torch.float32, "target"), C, T, d, w,
@@ -274,6 +344,13 @@ def reconstruct(bp: torch.Tensor, w: torch.Tensor, t: torch.Tensor, sets: torch.
                 used_w: Optional[torch.Tensor], t_draft: Optional[torch.Tensor],
                 status: torch.Tensor) -> None:
     n_items, C = bp.shape
+    _shape(w, (n_items,), "w")
+    _shape(t, (n_items,), "t")
+    _shape(sets, (C, (n_items + 63) // 64), "sets")
+    _shape(used_w, (C,), "used_w")
+    _shape(t_draft, (C,), "t_draft")
+    if status.numel() < 1:
+        raise KnapSpecError("status must hold one int32")
     _check(load().ks_reconstruct(_dev(bp, torch.uint8, "bp"), _dev(w, torch.int32, "w"),
                                  _dev(t, torch.float64, "t"), n_items, C,
                                  _dev(sets, torch.int64, "sets"),
@@ -285,6 +362,12 @@ def reconstruct(bp: torch.Tensor, w: torch.Tensor, t: torch.Tensor, sets: torch.
 def tpt_argmax(values: torch.Tensor, t_draft: torch.Tensor, t_target: float, prm: Params,
                tpt: Optional[torch.Tensor], best: torch.Tensor,
                best_tpt: Optional[torch.Tensor]) -> None:
+    C = values.numel()
+    _shape(t_draft, (C,), "t_draft")
+    _shape(tpt, (C, prm.gamma_max), "tpt")
+    _shape(best, (2,), "best")
+    if best_tpt is not None and best_tpt.numel() < 1:
+        raise KnapSpecError("best_tpt must hold one float64")
     _check(load().ks_tpt_argmax(_dev(values, torch.float32, "values"),
                                 _dev(t_draft, torch.float64, "t_draft"), values.numel(),
                                 t_target, ctypes.byref(prm), _dev(tpt, torch.float64, "tpt"),
@@ -330,9 +413,9 @@ class Solver:
         self.model = model
         self.wdtype = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
         self._layers_keep = layers
-        self.layers = layer_array(layers, self.wdtype)
+        self.layers = layer_array(layers, self.wdtype, model)
         self._cache_keep = (k_cache, v_cache)
-        self.cache = cache_desc(k_cache, v_cache, ctx)
+        self.cache = cache_desc(k_cache, v_cache, ctx, model)
         self.T = T
         self.t = list(map(float, t))
         self.prm = prm
@@ -342,6 +425,7 @@ class Solver:
         self.w = list(w) if w is not None else quantize_weights(self.t, prm.n_bins)
         self.C = solve_cells(self.t, prm, self.w)
         self.ws = workspace(model, self.C, T, device)
+        self.device = self.ws.device
         C, n, words = self.C, self.n_items, (self.n_items + 63) // 64
         z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=device)
         self.out = SolveOutputs(
@@ -366,12 +450,17 @@ class Solver:
         self._w_arr = (ctypes.c_int32 * n)(*self.w)
 
     def solve(self, x0: torch.Tensor, ref: Optional[torch.Tensor] = None) -> SolveOutputs:
-        """Enqueue one solve on the current stream (results valid after a sync)."""
-        _check(load().ks_solve(ctypes.byref(self.model), self.layers, ctypes.byref(self.cache),
-                               self.T, _dev(x0, torch.float32, "x0"),
-                               _dev(ref, torch.float32, "ref"), self._w_arr, self._t_arr,
-                               ctypes.byref(self.prm), _dev(self.ws), self.ws.numel(),
-                               ctypes.byref(self.result), _stream()))
+        """Enqueue one solve on the current stream of the solver's device (results
+        valid after a sync)."""
+        _shape(x0, (self.T, self.model.d_model), "x0")
+        _shape(ref, (self.n_items + 1, self.T, self.model.d_model), "ref")
+        with torch.cuda.device(self.device):
+            _check(load().ks_solve(ctypes.byref(self.model), self.layers,
+                                   ctypes.byref(self.cache), self.T,
+                                   _dev(x0, torch.float32, "x0"),
+                                   _dev(ref, torch.float32, "ref"), self._w_arr, self._t_arr,
+                                   ctypes.byref(self.prm), _dev(self.ws), self.ws.numel(),
+                                   ctypes.byref(self.result), _stream()))
         return self.out
 
     def check_status(self) -> None:
@@ -406,6 +495,11 @@ def lemma_check(states: torch.Tensor, ref: torch.Tensor, lm_head: torch.Tensor,
     """Lemma 4.1 checker on N states [N][T][d] against ref [T][d] (see knapspec.h)."""
     N, T, d = states.shape
     V = lm_head.shape[0]
+    _shape(ref, (T, d), "ref")
+    _shape(lm_head, (V, d), "lm_head")
+    _shape(final_norm, (d,), "final_norm")
+    if status is not None and status.numel() < 1:
+        raise KnapSpecError("status must hold one int32")
     size = ctypes.c_size_t()
     _check(load().ks_lemma_workspace_size(N, T, d, V, ctypes.byref(size)))
     ws = torch.empty(size.value, dtype=torch.uint8, device=states.device)
