@@ -14,6 +14,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -91,26 +92,49 @@ def job_value(units_per_rank: float, ms_max: float, world: int) -> float:
 
 
 # ---------------------------------------------------------------- clocks
-class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+def pci_of(device: int):
+    """(domain, bus, device) PCI numbers of a CUDA device, or None if torch does not say."""
+    p = torch.cuda.get_device_properties(device)
+    try:
+        return (int(p.pci_domain_id), int(p.pci_bus_id), int(p.pci_device_id))
+    except AttributeError:
+        return None
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+
+def _parse_bus_id(text: str):
+    """nvidia-smi's "DDDDDDDD:BB:DD.F" -> (domain, bus, device), else None."""
+    m = re.fullmatch(r"\s*([0-9A-Fa-f]+):([0-9A-Fa-f]+):([0-9A-Fa-f]+)\.[0-9A-Fa-f]+\s*", text)
+    return tuple(int(g, 16) for g in m.groups()) if m else None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region.
+
+    Every GPU nvidia-smi lists is sampled; the summary keeps the rows of the
+    GPU whose PCI address is `pci` (the CUDA device's), else -- when the
+    address is unknown or not listed -- the only GPU listed, else the one at
+    nvidia-smi index `gpu_index`."""
+
+    FIELDS = ("pci.bus_id,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pci=None):
         self.idx = gpu_index
+        self.pci = pci
         self.proc = None
         self.path = None
+        self.out = None
 
     def __enter__(self):
         import tempfile
         fd, self.path = tempfile.mkstemp(prefix="ks_clocks_", suffix=".csv")
         os.close(fd)
+        self.out = open(self.path, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.idx), "-lms", "200"], stdout=open(self.path, "w"),
+                 "-lms", "200"], stdout=self.out,
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -124,27 +148,44 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+                self.proc.wait(timeout=5)
+        if self.out is not None:
+            self.out.close()
 
     def summary(self):
+        """Median SM clock, max clock and the throttle reasons seen; removes the samples file."""
         if self.proc is None or not self.path or not os.path.exists(self.path):
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = {}                              # bus id text -> (nvidia-smi index, field rows)
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
+            rows.setdefault(f[0], (f[1], []))[1].append(f)
+        os.unlink(self.path)
+        pick = [k for k in rows if self.pci is not None and _parse_bus_id(k) == tuple(self.pci)]
+        if not pick and len(rows) == 1:
+            pick = list(rows)
+        if not pick:
+            pick = [k for k, (idx, _) in rows.items() if idx == str(self.idx)]
+        if not pick:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": ["no nvidia-smi samples of this GPU"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for f in rows[pick[0]][1]:
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                sm.append(float(f[2]))
+                smax = float(f[3])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
-        os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "reasons": sorted(reasons), "gpu": pick[0]}
 
 
 def load_peaks():
@@ -261,7 +302,8 @@ def run_ours(args, rank, world, local):
     x0 = inp.x0
     stream = torch.cuda.current_stream()
 
-    for _ in range(max(3, args.warmup)):
+    warmup = max(3, args.warmup)               # at least three untimed solves
+    for _ in range(warmup):
         solver.solve(x0)
     torch.cuda.synchronize()
     solver.check_status()
@@ -271,7 +313,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, pci_of(local)) as clk:
         B.profile_start(timing=True)
         e0.record(stream)
         for _ in range(args.steps):
@@ -279,6 +321,7 @@ def run_ours(args, rank, world, local):
         e1.record(stream)
         torch.cuda.synchronize()
         stats = B.profile_stop()
+    clocks = clk.summary()                     # every rank removes its own samples file
     barrier(world)
     solver.check_status()
     ms = e0.elapsed_time(e1) / args.steps
@@ -373,7 +416,7 @@ def run_ours(args, rank, world, local):
     if rank == 0:
         cfg = base_config(wl, C, world)
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "steps": args.steps, "warmup": warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if wl.wdtype == "bf16" else "f32", "data": "synthetic",
                 "config": cfg,
@@ -392,7 +435,7 @@ def run_ours(args, rank, world, local):
                                         "ms_per_step": s["total_ms"] / args.steps,
                                         "share": s["total_ms"] / max(1e-9, sum(x["total_ms"] for x in stats))}
                             for s in stats},
-                "clocks": clk.summary()}
+                "clocks": clocks}
         print(json.dumps(line), flush=True)
 
 
