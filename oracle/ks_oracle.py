@@ -42,6 +42,11 @@ R6 the compared state is the residual stream right after item i.
 R7 a candidate's queries attend over the full model's cached keys/values of
    all ctx+T positions (the evaluation tokens are already verified); token t
    sees positions <= ctx + t.  Wk/Wv are not used by the DP.
+R7w the alternative, ``kv="window"``: the keys/values of the T window
+   positions ctx .. ctx+T-1 are recomputed from the candidate's own normalised
+   state through the layer's Wk/Wv (keys rotated at their positions); positions
+   0 .. ctx-1 still come from the full model's cache.  Token t sees the same
+   positions as under R7.
 R8 RoPE is the rotate-half form, theta_j = base^(-2j/hd), position ctx + t;
    only the candidate's queries are rotated (the cache holds rotated keys).
 R9 RMSNorm y = x / sqrt(mean(x^2) + eps) * g.
@@ -99,8 +104,9 @@ class Model:
 
     ``layers[l]`` maps attn_norm [d], wq [Hq*hd][d], wo [d][Hq*hd], mlp_norm [d],
     w_gate [F][d], w_up [F][d], w_down [d][F] to arrays (any float dtype; they
-    are widened to fp64 where used).  ``k_cache``/``v_cache`` are sequences over
-    layers of [n_pos][Hkv][hd] arrays.
+    are widened to fp64 where used), and -- only for reading R7w -- wk and wv
+    [Hkv*hd][d].  ``k_cache``/``v_cache`` are sequences over layers of
+    [n_pos][Hkv][hd] arrays.
     """
 
     n_q_heads: int
@@ -179,15 +185,44 @@ def attention_core(q: np.ndarray, k: np.ndarray, v: np.ndarray, ctx: int,
     return out
 
 
-def attn_item(model: Model, layer: int, H: np.ndarray, ctx: int) -> np.ndarray:
-    """Attention sublayer on states H [M, T, d]: H + Attn(RMSNorm(H)) (R6-R9)."""
+def window_kv(model: Model, layer: int, xh: np.ndarray, ctx: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Keys and values of the T window positions from normalised states xh [M, T, d]
+    (reading R7w): k = RoPE(xh Wk^T) at positions ctx + t, v = xh Wv^T; each
+    [M, T, Hkv, hd]."""
+    Lw = model.layers[layer]
+    M, T, d = xh.shape
+    shape = (M, T, model.n_kv_heads, model.head_dim)
+    k = (xh.reshape(M * T, d) @ np.asarray(Lw["wk"], F64).T).reshape(shape)
+    k = rope_rotate_half(k, ctx + np.arange(T), model.rope_base)
+    v = (xh.reshape(M * T, d) @ np.asarray(Lw["wv"], F64).T).reshape(shape)
+    return k, v
+
+
+def attn_item(model: Model, layer: int, H: np.ndarray, ctx: int, kv: str = "cache") -> np.ndarray:
+    """Attention sublayer on states H [M, T, d]: H + Attn(RMSNorm(H)) (R6-R9).
+
+    ``kv="cache"`` reads every key/value from the full model's cache (R7);
+    ``kv="window"`` replaces the window positions' keys/values by the
+    candidate's own (R7w), so each state attends over its own key set.
+    """
     Lw = model.layers[layer]
     M, T, d = H.shape
     xh = rms_norm(H, Lw["attn_norm"], model.rms_eps)
     q = xh.reshape(M * T, d) @ np.asarray(Lw["wq"], F64).T
     q = q.reshape(M, T, model.n_q_heads, model.head_dim)
     q = rope_rotate_half(q, ctx + np.arange(T), model.rope_base)
-    o = attention_core(q, model.k_cache[layer], model.v_cache[layer], ctx, model.n_kv_heads)
+    if kv == "cache":
+        o = attention_core(q, model.k_cache[layer], model.v_cache[layer], ctx, model.n_kv_heads)
+    elif kv == "window":
+        kw, vw = window_kv(model, layer, xh, ctx)
+        kc = np.asarray(model.k_cache[layer][:ctx], F64)
+        vc = np.asarray(model.v_cache[layer][:ctx], F64)
+        o = np.concatenate([
+            attention_core(q[m:m + 1], np.concatenate([kc, kw[m]]), np.concatenate([vc, vw[m]]),
+                           ctx, model.n_kv_heads)
+            for m in range(M)])
+    else:
+        raise ValueError(kv)
     y = o.reshape(M * T, -1) @ np.asarray(Lw["wo"], F64).T
     return H + y.reshape(M, T, d)
 
@@ -204,31 +239,34 @@ def mlp_item(model: Model, layer: int, H: np.ndarray) -> np.ndarray:
     return H + y.reshape(M, T, d)
 
 
-def apply_item(model: Model, k: int, H: np.ndarray, ctx: int, per_cell: bool = False) -> np.ndarray:
+def apply_item(model: Model, k: int, H: np.ndarray, ctx: int, per_cell: bool = False,
+               kv: str = "cache") -> np.ndarray:
     """Item k (2l = Attention of layer l, 2l+1 = MLP of layer l) on H [M, T, d].
 
     With ``per_cell`` each of the M states goes through its own call, so every
     state sees exactly the arithmetic of a single-state call (used where a
-    bit-for-bit comparison with the reference chain is wanted).
+    bit-for-bit comparison with the reference chain is wanted).  ``kv`` picks
+    reading R7 ("cache") or R7w ("window") for the Attention items.
     """
     H = np.asarray(H, F64)
     if per_cell and H.shape[0] > 1:
-        return np.concatenate([apply_item(model, k, H[m:m + 1], ctx) for m in range(H.shape[0])])
+        return np.concatenate([apply_item(model, k, H[m:m + 1], ctx, kv=kv)
+                               for m in range(H.shape[0])])
     layer = k // 2
     if k % 2 == 0:
-        return attn_item(model, layer, H, ctx)
+        return attn_item(model, layer, H, ctx, kv=kv)
     return mlp_item(model, layer, H)
 
 
 # --------------------------------------------------------------------------
 # a1: reference states; value function
 # --------------------------------------------------------------------------
-def reference_states(model: Model, x0: np.ndarray, ctx: int) -> np.ndarray:
+def reference_states(model: Model, x0: np.ndarray, ctx: int, kv: str = "cache") -> np.ndarray:
     """X^(0) = x0 and X^(k+1) = item_k(X^(k)) for the full model: [2L+1, T, d]."""
     x = np.asarray(x0, F64)[None]
     out = [x[0]]
     for k in range(model.n_items):
-        x = apply_item(model, k, x, ctx)
+        x = apply_item(model, k, x, ctx, kv=kv)
         out.append(x[0])
     return np.stack(out)
 
@@ -361,7 +399,7 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
              per_cell: bool = False, ref: Optional[np.ndarray] = None,
              alpha_lo: float = 0.5, alpha_scale: float = 0.5, alpha_max: float = 0.99,
              keep_states: bool = False, prune_tau: Optional[float] = None,
-             skip_cap: Optional[int] = None) -> Solve:
+             skip_cap: Optional[int] = None, kv: str = "cache") -> Solve:
     """KnapSpec's DP over all budget cells, reconstruction and TPT selection.
 
     ``n_cells`` < K+1 computes only the budgets 0 .. n_cells-1, which equal the
@@ -375,6 +413,9 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
     review's "Reading between the lines"; reading R16).  A dropped cell is
     invalid: its value is NaN, no later candidate reads it, and a final
     invalid cell has no set.
+
+    ``kv`` picks the attention's key/value reading for every item, the
+    reference chain included: R7 ("cache") or R7w ("window").
     """
     x0 = np.asarray(x0, F64)
     n_items = model.n_items
@@ -383,7 +424,7 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
     K = int(sum(int(x) for x in w))
     C = K + 1 if n_cells is None else int(n_cells)
     if ref is None:
-        ref = reference_states(model, x0, ctx)
+        ref = reference_states(model, x0, ctx, kv=kv)
     T, d = x0.shape
     init = np.broadcast_to(x0, (C, T, d)).copy()
     if mode == "at_most":
@@ -395,7 +436,7 @@ def dp_solve(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], t: Sequen
         raise ValueError(mode)
 
     dp = knapsack_dp(w, C, init, init_valid,
-                     lambda k, H: apply_item(model, k, H, ctx, per_cell=per_cell),
+                     lambda k, H: apply_item(model, k, H, ctx, per_cell=per_cell, kv=kv),
                      lambda r, H: meancos(H, ref[r]),
                      prune=pruning_rule(w, C, prune_tau, skip_cap))
     sets, used = [], np.zeros(C, dtype=np.int64)
@@ -502,25 +543,26 @@ def tpt_argmax(grid: np.ndarray) -> Tuple[int, int, float]:
 # Checks that use the same pieces: re-running a set, exhaustive search
 # --------------------------------------------------------------------------
 def chain(model: Model, x0: np.ndarray, ctx: int, items: Sequence[int],
-          upto: Optional[int] = None) -> np.ndarray:
+          upto: Optional[int] = None, kv: str = "cache") -> np.ndarray:
     """Run the executed items (in order) on x0; items >= upto are ignored."""
     x = np.asarray(x0, F64)[None]
     n = model.n_items if upto is None else upto
     for k in range(n):
         if k in items:
-            x = apply_item(model, k, x, ctx)
+            x = apply_item(model, k, x, ctx, kv=kv)
     return x[0]
 
 
 def eval_set(model: Model, x0: np.ndarray, ctx: int, items: Sequence[int],
-             ref: np.ndarray, upto: Optional[int] = None) -> float:
+             ref: np.ndarray, upto: Optional[int] = None, kv: str = "cache") -> float:
     """Value of a layer set re-run from scratch: meancos(chain(x0), X^(upto))."""
     n = model.n_items if upto is None else upto
-    return float(meancos(chain(model, x0, ctx, set(items), n)[None], ref[n])[0])
+    return float(meancos(chain(model, x0, ctx, set(items), n, kv=kv)[None], ref[n])[0])
 
 
 def brute_force(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], ref: np.ndarray,
-                n_items: Optional[int] = None) -> Tuple[np.ndarray, List[Tuple[int, ...]]]:
+                n_items: Optional[int] = None,
+                kv: str = "cache") -> Tuple[np.ndarray, List[Tuple[int, ...]]]:
     """Best value over all subsets of the first n_items items for every budget b.
 
     best[b] = max over S with sum(w_S) <= b of meancos(chain_S(x0), X^(n_items)):
@@ -542,7 +584,8 @@ def brute_force(model: Model, x0: np.ndarray, ctx: int, w: Sequence[int], ref: n
                 arg[used] = chosen
             return
         visit(k + 1, state, used, chosen)
-        visit(k + 1, apply_item(model, k, state[None], ctx)[0], used + int(w[k]), chosen + (k,))
+        visit(k + 1, apply_item(model, k, state[None], ctx, kv=kv)[0], used + int(w[k]),
+              chosen + (k,))
 
     visit(0, x0, 0, ())
     # "at most b": running maximum over budgets
