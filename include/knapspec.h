@@ -334,6 +334,29 @@ KS_API ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* la
                    const int32_t* w, const double* t, const ks_params* params,
                    void* workspace, size_t workspace_bytes, ks_result* out, ks_stream_t stream);
 
+/*
+ * Re-run check of one layer set (review: the DP keeps a single state per cell
+ * with no optimality proof, referee major 1 on Eq. 8 / Algorithm 1 -- so a
+ * chosen set is worth checking from scratch): the set's items run on x0 in
+ * increasing item order, each exactly as ks_sublayer_forward runs it on one
+ * state, and the result is scored against target:
+ *   value = meancos(state, target), as ks_select_step scores a skip candidate.
+ * With target = X^(2L) (ks_result.ref_states row n_items) and the set of cell
+ * b, value reproduces ks_result.values[b] up to the rounding of the
+ * normalised operand (the solve fuses that RMSNorm into its select step).
+ * set: HOST [words] bitmask, bit k = item k runs (bits >= n_items must be 0).
+ * x0, target: device [T][d] fp32.  value_out: device [1] fp32.  state_out:
+ * device [T][d] fp32 (the set's final state) or NULL.  The workspace must hold
+ * ks_workspace_size(model, 1, T); its status word reports a timed-out wait
+ * (ks_workspace_status).  Errors: as ks_sublayer_forward, and
+ * KS_ERR_INVALID_ARG for a NULL argument or a bit at or above n_items.
+ */
+KS_API ks_status ks_eval_set(const ks_model_desc* model, const ks_layer_weights* layers,
+                             const ks_cache_desc* cache, int32_t T, const float* x0,
+                             const float* target, const uint64_t* set, float* value_out,
+                             float* state_out, void* workspace, size_t workspace_bytes,
+                             ks_stream_t stream);
+
 /* C = sum(w) + 1 for the weights ks_solve would use (w, or t quantised with
  * params->n_bins when w is NULL).  Host only. */
 KS_API ks_status ks_solve_cells(int32_t n_items, const int32_t* w, const double* t,

@@ -74,7 +74,7 @@ EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weigh
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
            "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
            "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16",
-           "ks_check_bounded_wait", "ks_lemma_workspace_size", "ks_lemma_check"]
+           "ks_check_bounded_wait", "ks_lemma_workspace_size", "ks_lemma_check", "ks_eval_set"]
 
 _lib = None
 
@@ -112,6 +112,7 @@ def load() -> ctypes.CDLL:
                            ctypes.c_int),
         "ks_attention_bf16": ([P, P, P, I64, I32, I32, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
+        "ks_eval_set": ([P, P, P, I32, P, P, P, P, P, P, SZ, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -275,6 +276,34 @@ def reference_forward_noalloc(model: ModelDesc, layers, cache: CacheDesc, T: int
                                                T, _dev(x0, torch.float32, "x0"),
                                                _dev(ref_out, torch.float32, "ref_out"),
                                                _stream()))
+
+
+def set_mask(items: Sequence[int], n_items: int):
+    """Host bitmask of a layer set (bit k = item k), as ks_eval_set takes it."""
+    words = (ctypes.c_uint64 * ((n_items + 63) // 64))()
+    for k in items:
+        if not 0 <= int(k) < n_items:
+            raise KnapSpecError(f"item {k} is outside 0 .. {n_items - 1}")
+        words[int(k) >> 6] |= 1 << (int(k) & 63)
+    return words
+
+
+def eval_set(model: ModelDesc, layers, cache: CacheDesc, T: int, x0: torch.Tensor,
+             target: torch.Tensor, items: Sequence[int], ws: torch.Tensor,
+             value_out: torch.Tensor, state_out: Optional[torch.Tensor] = None) -> None:
+    """Run only the given items on x0 and score the state against target
+    (ks_eval_set): value_out [1] = meancos(state, target); state_out [T][d]."""
+    d = model.d_model
+    _shape(x0, (T, d), "x0")
+    _shape(target, (T, d), "target")
+    _shape(value_out, (1,), "value_out")
+    _shape(state_out, (T, d), "state_out")
+    mask = set_mask(items, 2 * model.n_layers)
+    _check(load().ks_eval_set(ctypes.byref(model), layers, ctypes.byref(cache), T,
+                              _dev(x0, torch.float32, "x0"), _dev(target, torch.float32, "target"),
+                              mask, _dev(value_out, torch.float32, "value_out"),
+                              _dev(state_out, torch.float32, "state_out"),
+                              _dev(ws, name="workspace"), ws.numel(), _stream()))
 
 
 def workspace_status(ws: torch.Tensor) -> int:

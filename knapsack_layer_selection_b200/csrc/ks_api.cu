@@ -585,6 +585,38 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   return KS_OK;
 }
 
+ks_status ks_eval_set(const ks_model_desc* model, const ks_layer_weights* layers,
+                      const ks_cache_desc* cache, int32_t T, const float* x0, const float* target,
+                      const uint64_t* set, float* value_out, float* state_out, void* workspace,
+                      size_t workspace_bytes, ks_stream_t stream) {
+  Ctx c;
+  KS_TRY(make_ctx(model, layers, cache, T, 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
+  if (!x0 || !target || !set || !value_out) return fail(KS_ERR_INVALID_ARG, "eval_set: NULL argument");
+  const int n_items = 2 * model->n_layers;
+  const int words = (n_items + 63) / 64;
+  if (n_items % 64 && (set[words - 1] >> (n_items % 64)) != 0)
+    return fail(KS_ERR_INVALID_ARG, "eval_set: the set has bits at or above n_items");
+  const long long cell = (long long)T * model->d_model;
+  KS_CUDA_TRY(cudaMemsetAsync(c.status, 0, sizeof(int32_t), c.st));
+  KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
+  // the set's items in increasing order on x0, each exactly as ks_sublayer_forward runs it
+  float* a = c.ws.prev;
+  float* b = c.ws.cur;
+  KS_CUDA_TRY(cudaMemcpyAsync(a, x0, cell * sizeof(float), cudaMemcpyDeviceToDevice, c.st));
+  for (int k = 0; k < n_items; ++k) {
+    if (!((set[k >> 6] >> (k & 63)) & 1)) continue;
+    KS_TRY(sublayer(c, k, a, 1, b));
+    std::swap(a, b);
+  }
+  // value: the select step's skip score of one cell (C = 1 < w, so no execute
+  // candidate is read); the copy of the kept state goes to scratch
+  KS_TRY(launch_select(a, a, target, 1, T, model->d_model, 1, c.ws.exec, value_out, c.ws.bp,
+                       nullptr, nullptr, c.st));
+  if (state_out)
+    KS_CUDA_TRY(cudaMemcpyAsync(state_out, a, cell * sizeof(float), cudaMemcpyDeviceToDevice, c.st));
+  return KS_OK;
+}
+
 ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
                                        const ks_layer_weights* layers,
                                        const ks_cache_desc* cache, int32_t T, const float* x0,

@@ -157,3 +157,41 @@ def test_step_calls_reject_bad_arguments(lib):
     prm = B.params(0, 8)
     st = lib.ks_tpt_argmax(p, p, 4, 10.0, ctypes.byref(prm), None, p, None, None)
     assert st == 1   # gamma_max must be >= 1
+
+
+def test_eval_set_rejects_bad_arguments_before_any_launch(lib):
+    """ks_eval_set checks its model, cache, workspace, pointers and set bits on
+    the host; nothing here reaches the device (the pointers are never read)."""
+    m = B.model_desc(3, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")        # 6 items
+    layers = (B.LayerWeights * 3)()
+    for i in range(3):
+        for f, _ in B.LayerWeights._fields_:
+            setattr(layers[i], f, 256)
+    cache = B.CacheDesc(256, 256, 16, 8)
+    p = ctypes.c_void_p(256)
+    need = B.workspace_size(m, 1, 4)
+    ok_set = B.set_mask([0, 3, 5], 6)
+    # NULL x0
+    st = lib.ks_eval_set(ctypes.byref(m), layers, ctypes.byref(cache), 4, None, p, ok_set, p,
+                         None, p, need, None)
+    assert st == 1 and b"NULL" in lib.ks_last_error()
+    # a bit above the model's items
+    bad_set = (ctypes.c_uint64 * 1)(1 << 6)
+    st = lib.ks_eval_set(ctypes.byref(m), layers, ctypes.byref(cache), 4, p, p, bad_set, p,
+                         None, p, need, None)
+    assert st == 1 and b"n_items" in lib.ks_last_error()
+    # a workspace far too small (every case here must stop before a device call:
+    # the pointers are not device memory)
+    st = lib.ks_eval_set(ctypes.byref(m), layers, ctypes.byref(cache), 4, p, p, ok_set, p,
+                         None, p, 1024, None)
+    assert st == 3 and b"workspace" in lib.ks_last_error()
+    # cache too short for ctx + T
+    short = B.CacheDesc(256, 256, 11, 8)
+    st = lib.ks_eval_set(ctypes.byref(m), layers, ctypes.byref(short), 4, p, p, ok_set, p,
+                         None, p, need, None)
+    assert st == 1 and b"cache_rows" in lib.ks_last_error()
+    # the binding's mask: one bit per item, items outside the model refused
+    assert list(B.set_mask([0, 3, 5], 6)) == [0b101001]
+    assert list(B.set_mask([64, 1], 70)) == [2, 1]
+    with pytest.raises(B.KnapSpecError, match="outside"):
+        B.set_mask([6], 6)
