@@ -75,7 +75,11 @@ typedef enum {
 typedef enum { KS_F32 = 0, KS_BF16 = 1 } ks_dtype;
 
 /* Decoder shape.  head_dim must be 64 or 128; n_q_heads a multiple of
- * n_kv_heads; d_model a multiple of 64; ffn a multiple of 16. */
+ * n_kv_heads; d_model a multiple of 64; ffn a multiple of 16.  bf16 weights
+ * run on the tensor-core GEMM, whose output tiles are 256 columns wide (128
+ * for the SwiGLU gate/up pair): there d_model and n_q_heads * head_dim must
+ * be multiples of 256 and ffn of 128 (else KS_ERR_UNSUPPORTED, before any
+ * launch). */
 typedef struct {
   int32_t n_layers;
   int32_t d_model;

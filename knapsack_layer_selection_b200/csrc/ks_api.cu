@@ -44,6 +44,13 @@ static ks_status check_model(const ks_model_desc* m) {
   if (m->wdtype != KS_F32 && m->wdtype != KS_BF16) return fail(KS_ERR_INVALID_ARG, "wdtype");
   if (!(m->rms_eps >= 0.f)) return fail(KS_ERR_INVALID_ARG, "rms_eps must be >= 0");
   if (!(m->rope_base > 0.0)) return fail(KS_ERR_INVALID_ARG, "rope_base must be > 0");
+  if (m->wdtype == KS_BF16) {
+    // the tensor-core GEMM's output tiles: 256 columns (Q, O, down), 128 (gate/up)
+    if (m->d_model % 256 || (m->n_q_heads * m->head_dim) % 256)
+      return fail(KS_ERR_UNSUPPORTED,
+                  "bf16 weights: d_model and n_q_heads * head_dim must be multiples of 256");
+    if (m->ffn % 128) return fail(KS_ERR_UNSUPPORTED, "bf16 weights: ffn must be a multiple of 128");
+  }
   return KS_OK;
 }
 

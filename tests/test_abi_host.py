@@ -103,6 +103,14 @@ def test_model_checks(lib):
     good = B.model_desc(2, 128, 4, 4, 64, 128, 1e-6, 1e4, "f32")
     with pytest.raises(B.KnapSpecError, match="T must"):
         B.workspace_size(good, 10, 0)
+    # bf16 runs on the tensor-core GEMM: its tile widths are checked up front
+    assert B.workspace_size(B.model_desc(2, 512, 4, 2, 64, 384, 1e-6, 1e4, "bf16"), 10, 4) > 0
+    for d, hq, ffn in ((320, 4, 384), (512, 3, 384), (512, 4, 320)):
+        bad = B.model_desc(2, d, hq, 1, 64, ffn, 1e-6, 1e4, "bf16")
+        with pytest.raises(B.KnapSpecError, match="bf16 weights"):
+            B.workspace_size(bad, 10, 4)
+    # the same shapes are fine with fp32 weights (SIMT kernels)
+    assert B.workspace_size(B.model_desc(2, 320, 4, 1, 64, 320, 1e-6, 1e4, "f32"), 10, 4) > 0
 
 
 def test_solve_rejects_null_and_short_workspace_before_any_launch(lib):
