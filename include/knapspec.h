@@ -109,7 +109,9 @@ typedef struct {
 /* The full model's KV cache (device, dtype = wdtype), laid out
  * [n_layers][cache_rows][n_kv_heads][head_dim] for K and for V, keys already
  * rotated.  Evaluation token t (0 .. T-1) sits at position ctx + t and attends
- * to positions 0 .. ctx + t, so cache_rows >= ctx + T. */
+ * to positions 0 .. ctx + t, so cache_rows >= ctx + T.  With fp32 weights
+ * (SIMT kernels) ctx + T + head_dim must be at most 51200, else
+ * KS_ERR_UNSUPPORTED before any launch. */
 typedef struct {
   const void* k_cache;
   const void* v_cache;

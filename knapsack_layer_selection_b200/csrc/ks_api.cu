@@ -64,7 +64,9 @@ static ks_status check_cache(const ks_model_desc* m, const ks_cache_desc* c, int
   if (c->ctx < 0) return fail(KS_ERR_INVALID_ARG, "ctx must be >= 0");
   if (c->cache_rows < (int64_t)c->ctx + T)
     return fail(KS_ERR_INVALID_ARG, "cache_rows must be >= ctx + T");
-  (void)m;
+  // fp32 weights run the SIMT attention, which keeps a row's scores in shared memory
+  if (m->wdtype == KS_F32 && (int64_t)m->head_dim + c->ctx + T > 51200)
+    return fail(KS_ERR_UNSUPPORTED, "fp32 weights: ctx + T + head_dim must be at most 51200");
   return KS_OK;
 }
 

@@ -143,6 +143,27 @@ def test_solve_rejects_null_and_short_workspace_before_any_launch(lib):
     assert st == 1 and b"cache_rows" in lib.ks_last_error()
 
 
+def test_fp32_context_limit_is_checked_before_any_launch(lib):
+    """fp32 weights run the SIMT attention, whose scores of one row live in
+    shared memory: a context beyond it is refused on the host."""
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    layers = (B.LayerWeights * 1)()
+    for f, _ in B.LayerWeights._fields_:
+        setattr(layers[0], f, 256)
+    p = ctypes.c_void_p(256)
+    T = 4
+    too_long = B.CacheDesc(256, 256, 60000, 51200 - 64 - T + 1)
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(too_long), T, 0, p, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 2 and b"51200" in lib.ks_last_error()
+    # one position less passes the cache check and stops at the next host check
+    # (a NULL state pointer), still before any launch
+    fits = B.CacheDesc(256, 256, 60000, 51200 - 64 - T)
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(fits), T, 0, None, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 1 and b"states" in lib.ks_last_error()
+
+
 def test_solve_rejects_unknown_budget_mode(lib):
     m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
     prm = B.params(4, 8)
