@@ -31,7 +31,10 @@
  *  - Pointers named "device" are CUDA device pointers (cudaMalloc or a
  *    torch CUDA tensor); "host" pointers are ordinary host memory.  The caller
  *    owns every buffer; the library allocates nothing.  All dense arrays are
- *    row-major and contiguous.
+ *    row-major and contiguous.  Device arrays of weights, caches and states
+ *    (and the GEMM / attention utilities' operands and outputs) must start on
+ *    a 16-byte boundary: the kernels move them 16 bytes at a time.  A
+ *    misaligned pointer is KS_ERR_INVALID_ARG, before anything is enqueued.
  *  - Calls that take a stream are asynchronous on it: they validate their
  *    arguments on the host, enqueue kernels and return.  Results are valid
  *    once the stream has been synchronised.  Host-side argument errors return

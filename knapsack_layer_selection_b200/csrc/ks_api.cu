@@ -61,6 +61,7 @@ static ks_status check_T(int T) {
 
 static ks_status check_cache(const ks_model_desc* m, const ks_cache_desc* c, int T) {
   if (!c || !c->k_cache || !c->v_cache) return fail(KS_ERR_INVALID_ARG, "cache is NULL");
+  KS_TRY(check_aligned16({c->k_cache, c->v_cache}, "cache"));
   if (c->ctx < 0) return fail(KS_ERR_INVALID_ARG, "ctx must be >= 0");
   if (c->cache_rows < (int64_t)c->ctx + T)
     return fail(KS_ERR_INVALID_ARG, "cache_rows must be >= ctx + T");
@@ -76,6 +77,8 @@ static ks_status check_layers(const ks_model_desc* m, const ks_layer_weights* la
     const ks_layer_weights& L = layers[l];
     if (!L.attn_norm || !L.wq || !L.wo || !L.mlp_norm || !L.w_gate || !L.w_up || !L.w_down)
       return fail(KS_ERR_INVALID_ARG, "layer " + std::to_string(l) + " has a NULL weight");
+    KS_TRY(check_aligned16({L.attn_norm, L.wq, L.wo, L.mlp_norm, L.w_gate, L.w_up, L.w_down},
+                           "layer weights"));
   }
   return KS_OK;
 }
@@ -395,6 +398,7 @@ ks_status ks_sublayer_forward(const ks_model_desc* model, const ks_layer_weights
   if (item < 0 || item >= 2 * model->n_layers) return fail(KS_ERR_INVALID_ARG, "item out of range");
   if (E < 0) return fail(KS_ERR_INVALID_ARG, "E must be >= 0");
   if (E > 0 && (!states_in || !states_out)) return fail(KS_ERR_INVALID_ARG, "states are NULL");
+  KS_TRY(check_aligned16({states_in, states_out}, "sublayer_forward"));
   KS_CUDA_TRY(cudaMemsetAsync(c.status, 0, sizeof(int32_t), c.st));
   KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
   return sublayer(c, item, states_in, E, states_out);
@@ -407,6 +411,7 @@ ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer_weight
   Ctx c;
   KS_TRY(make_ctx(model, layers, cache, T, 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
   if (!x0 || !ref_out) return fail(KS_ERR_INVALID_ARG, "x0 / ref_out is NULL");
+  KS_TRY(check_aligned16({x0, ref_out}, "reference_forward"));
   KS_CUDA_TRY(cudaMemsetAsync(c.status, 0, sizeof(int32_t), c.st));
   KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, c.st));
   return reference_chain(c, x0, ref_out);
@@ -419,6 +424,7 @@ ks_status ks_select_step(const float* prev, const float* exec, const float* targ
   if (C < 1 || T < 1 || d < 4 || w < 1) return fail(KS_ERR_INVALID_ARG, "select: C, T >= 1, d >= 4, w >= 1");
   if (C > w && !exec) return fail(KS_ERR_INVALID_ARG, "select: exec is NULL");
   if (prev == cur) return fail(KS_ERR_INVALID_ARG, "select: prev and cur must differ");
+  KS_TRY(check_aligned16({prev, exec, target, cur}, "select"));
   return launch_select(prev, exec, target, C, T, d, w, cur, val, bp, cos_skip, cos_exec,
                        (cudaStream_t)stream);
 }
@@ -485,6 +491,7 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     return fail(KS_ERR_INVALID_ARG, "solve: budget_mode must be KS_BUDGET_AT_MOST or KS_BUDGET_EXACT");
   if (params->prune_tau != params->prune_tau)
     return fail(KS_ERR_INVALID_ARG, "solve: prune_tau is NaN (use -INFINITY to turn it off)");
+  KS_TRY(check_aligned16({x0, ref, out->ref_states, out->final_states}, "solve"));
   const int n_items = 2 * model->n_layers;
   std::vector<int32_t> ww;
   KS_TRY(resolve_weights(n_items, w, t, params, &ww));
@@ -601,6 +608,7 @@ ks_status ks_eval_set(const ks_model_desc* model, const ks_layer_weights* layers
   Ctx c;
   KS_TRY(make_ctx(model, layers, cache, T, 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
   if (!x0 || !target || !set || !value_out) return fail(KS_ERR_INVALID_ARG, "eval_set: NULL argument");
+  KS_TRY(check_aligned16({x0, target}, "eval_set"));
   const int n_items = 2 * model->n_layers;
   const int words = (n_items + 63) / 64;
   if (n_items % 64 && (set[words - 1] >> (n_items % 64)) != 0)
@@ -635,6 +643,7 @@ ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
   KS_TRY(check_cache(model, cache, T));
   KS_TRY(check_layers(model, layers));
   if (!x0 || !ref_out) return fail(KS_ERR_INVALID_ARG, "x0 / ref_out is NULL");
+  KS_TRY(check_aligned16({x0, ref_out}, "reference_forward_noalloc"));
   Workspace w;
   const size_t need = carve_sublayer_only(model, T, nullptr, &w);
   if (need > kStaticScratchBytes)
@@ -661,6 +670,7 @@ ks_status ks_gemm_bf16(const void* A, const void* B, float* C, const float* resi
                        int32_t N, int32_t K, int32_t* status, ks_stream_t stream) {
   if (!A || !B || !C) return fail(KS_ERR_INVALID_ARG, "gemm: NULL pointer");
   if (M < 0 || N < 1 || K < 1) return fail(KS_ERR_INVALID_ARG, "gemm: bad size");
+  KS_TRY(check_aligned16({A, B, C, resid}, "gemm"));
   return tc_gemm(A, B, nullptr, C, resid, M, N, K, resid ? EPI_RESID_F32 : EPI_STORE_F32, nullptr,
                  1, 64, status, (cudaStream_t)stream);
 }
@@ -679,6 +689,7 @@ ks_status ks_attention_bf16(const void* q, const void* k_layer, const void* v_la
                             ks_stream_t stream) {
   if (!q || !k_layer || !v_layer || !out) return fail(KS_ERR_INVALID_ARG, "attention: NULL pointer");
   if (R < 0 || T < 1 || Hq < 1 || Hkv < 1 || ctx < 0) return fail(KS_ERR_INVALID_ARG, "attention: bad size");
+  KS_TRY(check_aligned16({q, k_layer, v_layer, out}, "attention"));
   return tc_attention(q, k_layer, v_layer, cache_rows, R, T, Hq, Hkv, head_dim, ctx, out, status,
                       (cudaStream_t)stream);
 }

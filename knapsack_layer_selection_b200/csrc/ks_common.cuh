@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <initializer_list>
 #include <string>
 
 #include "../../include/knapspec.h"
@@ -32,6 +33,16 @@ ks_status fail(ks_status s, const std::string& msg);
 #define KS_LAUNCH_CHECK() KS_CUDA_TRY(cudaGetLastError())
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Caller pointers that kernels move 16 bytes at a time (vector loads and
+// stores, TMA) must be 16-byte aligned; checked at the C ABI before any launch
+// so a misaligned view is an error code, not a misaligned access.  NULL passes.
+inline ks_status check_aligned16(std::initializer_list<const void*> ptrs, const char* call) {
+  for (const void* p : ptrs)
+    if (p && (reinterpret_cast<uintptr_t>(p) & 15))
+      return fail(KS_ERR_INVALID_ARG, std::string(call) + ": device pointers must be 16-byte aligned");
+  return KS_OK;
+}
 
 // Runs `set` (a function-attribute setup returning ks_status) once per device
 // for the call site owning `done`: function attributes are per device.  Two

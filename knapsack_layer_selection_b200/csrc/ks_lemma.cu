@@ -236,6 +236,7 @@ KS_API ks_status ks_lemma_check(const float* states, int32_t N, const float* ref
   if (d % 64 || d < 64) return fail(KS_ERR_UNSUPPORTED, "lemma: d must be a multiple of 64");
   if (V % 256 || V < 256) return fail(KS_ERR_UNSUPPORTED, "lemma: V must be a multiple of 256");
   if ((uintptr_t)workspace % 256) return fail(KS_ERR_INVALID_ARG, "lemma: workspace alignment");
+  KS_TRY(check_aligned16({states, ref, lm_head, final_norm}, "lemma"));
   const LemmaWs need = lemma_carve(N, T, d, V, nullptr);
   if (workspace_bytes < need.total) return fail(KS_ERR_WORKSPACE, "lemma: workspace too small");
   LemmaWs w = lemma_carve(N, T, d, V, (char*)workspace);

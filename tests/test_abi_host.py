@@ -224,3 +224,32 @@ def test_eval_set_rejects_bad_arguments_before_any_launch(lib):
     assert list(B.set_mask([64, 1], 70)) == [2, 1]
     with pytest.raises(B.KnapSpecError, match="outside"):
         B.set_mask([6], 6)
+
+
+def test_misaligned_device_pointers_are_refused_before_any_launch(lib):
+    """Kernels move caller data 16 bytes at a time (vector loads, TMA): a view
+    that starts off a 16-byte boundary is refused with an error code."""
+    p, q = ctypes.c_void_p(256), ctypes.c_void_p(256 + 4)
+    st = lib.ks_select_step(p, p, q, 4, 4, 64, 1, ctypes.c_void_p(512), p, p, None, None, None)
+    assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
+    st = lib.ks_gemm_bf16(p, p, q, None, 4, 256, 64, None, None)
+    assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
+    st = lib.ks_attention_bf16(p, p, p, 16, 4, 4, 2, 1, 64, 8, q, None, None)
+    assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
+    # a weight pointer of one layer, through the sublayer forward's model checks
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    layers = (B.LayerWeights * 1)()
+    for f, _ in B.LayerWeights._fields_:
+        setattr(layers[0], f, 256)
+    layers[0].w_up = 256 + 8
+    cache = B.CacheDesc(256, 256, 16, 8)
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(cache), 4, 0, p, 1, p, p,
+                                 1 << 40, None)
+    assert st == 1 and b"layer weights" in lib.ks_last_error()
+    # x0 of a solve
+    prm = B.params(4, 8)
+    t = (ctypes.c_double * 2)(1.0, 1.0)
+    res = B.Result(*([256] * 14))
+    st = lib.ks_solve(ctypes.byref(m), None, None, 4, q, None, None, t, ctypes.byref(prm), None, 0,
+                      ctypes.byref(res), None)
+    assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
