@@ -7,10 +7,11 @@
  * knapsack item whose integer weight is its latency (review, "What carries the
  * argument"; referee major 4 on §3.6).  For every latency-budget cell b the DP
  * keeps whichever of "skip item i" (carry cell b) and "execute item i" (run the
- * sublayer on cell b - w_i) has the higher cosine similarity to the full
- * model's hidden state X^(i) (Eq. 6-8, Algorithm 1; referee major 1), stores a
- * backpointer, reads one layer set per budget back (Algorithm 2; referee minor
- * 4) and grid-searches the draft length gamma for the largest Tokens-per-Time
+ * sublayer on cell b - w_i) scores higher, the score being the cosine with the
+ * state X^(i) the unpruned model reaches at that depth (Eq. 6-8, Algorithm 1;
+ * referee major 1), stores a backpointer, reads one layer set per budget back
+ * (Algorithm 2; referee minor 4) and grid-searches the draft length gamma for
+ * the largest Tokens-per-Time
  * TPT(S, gamma) = ((1 - a^(gamma+1)) / (1 - a)) / (gamma t_Draft(S) + t_Target)
  * (Eq. 4, Eq. 5).
  *

@@ -12,9 +12,9 @@ which paraphrases the paper's equations:
   weight is its (quantised) latency; Attention latency grows with the context
   length, MLP latency is flat ("What carries the argument"; referee major 4 on
   §3.6, w_Attn ~ t_Attn / Delta);
-* value -- cosine similarity of the draft hidden state to the full model's
-  reference hidden state X^(i) at the same depth (Eq. 6; referee major 1 on
-  §3.4 Eq. 8 / Algorithm 1);
+* value -- the cosine between a draft state and X^(i), the state the
+  unpruned model reaches at the same depth (Eq. 6; referee major 1 on §3.4
+  Eq. 8 / Algorithm 1);
 * recurrence -- one hidden state g[i, j] per (item, budget); it keeps whichever
   of "execute item i" and "skip item i" has the higher cosine to X^(i) (Eq. 7/8,
   Algorithm 1); one candidate layer set per budget is read back by walking the
