@@ -14,7 +14,7 @@ from scipy.spatial.distance import cosine as scipy_cosine
 from knapsack_layer_selection_b200 import workloads as W
 from oracle import ks_oracle as O
 from tests._util import oracle_model, x0_np
-from tests.test_oracle_pins import _states, _torch_attn_item, _torch_mlp_item
+from tests.test_oracle_pins import _lemma_case, _states, _torch_attn_item, _torch_mlp_item
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -180,3 +180,47 @@ def test_exact_mode_started_from_every_cell(tiny, monkeypatch):
     monkeypatch.setattr(O, "knapsack_dp", bad)
     s = O.dp_solve(m, x0_np(inp), wl.ctx, w, t, wl.gamma_max, mode="exact", per_cell=True)
     assert any(s.used_w[b] >= 0 and s.used_w[b] != b for b in range(len(s.values)))
+
+
+def test_lemma_distance_taken_as_the_nearest_row(monkeypatch):
+    """D is the largest ||w_i* - w_j||; the smallest one over j != i* breaks the
+    brute-force pin (and would make the bound claim more than it proves)."""
+    states, ref, Wm = _lemma_case(0)
+    good = O.lemma_check
+
+    def bad(states, ref, lm_head, final_gain, eps):
+        lc = good(states, ref, lm_head, final_gain, eps)
+        Wd = np.asarray(lm_head, O.F64)
+        lc.dist = np.array([np.min(np.linalg.norm(np.delete(Wd, i, 0) - Wd[i], axis=-1))
+                            for i in lc.istar])
+        return lc
+
+    monkeypatch.setattr(O, "lemma_check", bad)
+    lc = O.lemma_check(states, ref, Wm, None, 1e-6)
+    D = [max(np.linalg.norm(Wm[i] - Wm[j]) for j in range(len(Wm))) for i in lc.istar]
+    assert np.max(np.abs(lc.dist - np.array(D))) > 1e-6
+
+
+def test_lemma_without_the_equal_norm_rescale(monkeypatch):
+    """h' must be rescaled to ||h|| before ||h - h'|| is taken from the cosine;
+    without it the distance identity of the pins no longer holds."""
+    states, ref, Wm = _lemma_case(1)
+    good = O.lemma_check
+
+    def bad(states, ref, lm_head, final_gain, eps):
+        lc = good(states, ref, lm_head, final_gain, eps)
+        h = O.rms_norm(ref, np.ones(ref.shape[-1]), eps)
+        hp = O.rms_norm(states, np.ones(ref.shape[-1]), eps)        # not rescaled
+        nh = np.linalg.norm(h, axis=-1)
+        lc.cos = np.sum(hp * h[None], axis=-1) / (nh[None] * nh[None])
+        gap = np.sqrt(np.maximum(2.0 * nh[None] ** 2 * (1.0 - lc.cos), 0.0))
+        lc.slack = lc.margin[None] / lc.dist[None] - gap
+        return lc
+
+    monkeypatch.setattr(O, "lemma_check", bad)
+    lc = O.lemma_check(states, ref, Wm, None, 1e-6)
+    h = ref / np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True) + 1e-6)
+    hp = states / np.sqrt(np.mean(states ** 2, axis=-1, keepdims=True) + 1e-6)
+    hp = hp * (np.linalg.norm(h, axis=-1) / np.linalg.norm(hp, axis=-1))[..., None]
+    gap = np.linalg.norm(hp - h[None], axis=-1)
+    assert np.max(np.abs(gap - (lc.margin[None] / lc.dist[None] - lc.slack))) > 1e-6
