@@ -125,3 +125,22 @@ def test_model_shapes_of_weights_cache_and_states():
         B.reference_forward(m, None, None, T, _t(T, d), _t(wl.n_items, T, d), None)
     with pytest.raises(B.KnapSpecError, match="x0 must have shape"):
         B.reference_forward_noalloc(m, None, None, T, _t(T, d + 1), _t(wl.n_items + 1, T, d))
+
+
+def test_set_masks_round_trip_across_words():
+    """sets_to_lists reads the [C][words] bitmask ks_solve writes; set_mask
+    builds the one ks_eval_set takes.  Both agree with a plain bit walk,
+    including items past the first 64-bit word (the 32B shape has 128 items)."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for n in (1, 63, 64, 65, 128, 130):
+        words = (n + 63) // 64
+        lists = [sorted(rng.choice(n, size=int(rng.integers(0, n + 1)), replace=False).tolist())
+                 for _ in range(7)]
+        rows = np.zeros((len(lists), words), dtype=np.uint64)
+        for r, items in enumerate(lists):
+            mask = B.set_mask(items, n)
+            rows[r] = np.array(list(mask), dtype=np.uint64)
+            for k in range(n):
+                assert ((int(rows[r][k >> 6]) >> (k & 63)) & 1) == (k in items)
+        assert B.sets_to_lists(torch.from_numpy(rows.view(np.int64)), n) == lists
