@@ -98,8 +98,9 @@ typedef struct {
 
 /* Device pointers to one layer's weights (dtype = ks_model_desc.wdtype):
  * attn_norm [d], wq [Hq*hd][d], wo [d][Hq*hd], mlp_norm [d],
- * w_gate [ffn][d], w_up [ffn][d], w_down [d][ffn].
- * Wk/Wv are not needed: the DP reads keys and values from the cache. */
+ * w_gate [ffn][d], w_up [ffn][d], w_down [d][ffn]; wk, wv [Hkv*hd][d].
+ * wk and wv are read only under KS_KV_WINDOW (they may be NULL otherwise):
+ * with the default KS_KV_CACHE every key and value comes from the cache. */
 typedef struct {
   const void* attn_norm;
   const void* wq;
@@ -108,19 +109,38 @@ typedef struct {
   const void* w_gate;
   const void* w_up;
   const void* w_down;
+  const void* wk;
+  const void* wv;
 } ks_layer_weights;
+
+/* Where an Attention item's keys and values come from.  The review leaves the
+ * attention of a pruned draft's evaluation tokens open ("What carries the
+ * argument": the value compares a draft state with the full model's state,
+ * Eq. 6); two readings are offered:
+ *  KS_KV_CACHE  -- every position 0 .. ctx+T-1 from the full model's cache
+ *                  (the evaluation tokens are already verified tokens);
+ *  KS_KV_WINDOW -- positions 0 .. ctx-1 from the cache, and the T window
+ *                  positions' keys and values recomputed from the candidate
+ *                  state itself: k = RoPE(x^ Wk^T) at position ctx + t,
+ *                  v = x^ Wv^T, with x^ the item's normalised input.  Token t
+ *                  sees the context and window tokens 0 .. t of its own state.
+ * With bf16 weights (tensor-core kernels) KS_KV_WINDOW needs T to divide 128,
+ * so that a 128-row tile of the batch holds whole states. */
+typedef enum { KS_KV_CACHE = 0, KS_KV_WINDOW = 1 } ks_kv_mode;
 
 /* The full model's KV cache (device, dtype = wdtype), laid out
  * [n_layers][cache_rows][n_kv_heads][head_dim] for K and for V, keys already
  * rotated.  Evaluation token t (0 .. T-1) sits at position ctx + t and attends
  * to positions 0 .. ctx + t, so cache_rows >= ctx + T.  With fp32 weights
  * (SIMT kernels) ctx + T + head_dim must be at most 51200, else
- * KS_ERR_UNSUPPORTED before any launch. */
+ * KS_ERR_UNSUPPORTED before any launch.  kv_mode is a ks_kv_mode; under
+ * KS_KV_WINDOW the cache rows ctx .. ctx+T-1 are not read. */
 typedef struct {
   const void* k_cache;
   const void* v_cache;
   int64_t cache_rows;
   int32_t ctx;
+  int32_t kv_mode;
 } ks_cache_desc;
 
 /* Budget semantics of a cell b (the review notes the paper's main text and
@@ -150,8 +170,13 @@ typedef struct {
   int32_t skip_cap;
   /* Distinct-state execution: before each item, budget cells whose states are
    * bit-for-bit equal (and valid) are folded together and the item runs once
-   * per distinct state.  Results are identical to the dense solve (every row's
-   * arithmetic is independent of its batch); only the work shrinks.  0 = off. */
+   * per distinct state.  Candidates are found by a 64-bit fingerprint of each
+   * state and every fold is then confirmed by comparing the two states' bytes;
+   * a state whose bytes differ from its representative's runs on its own.
+   * Results are therefore identical to the dense solve (every row's arithmetic
+   * is independent of its batch); only the work shrinks.  0 = off, 1 = on,
+   * 2 = on with the fingerprints cut to 8 bits, so that unequal states collide
+   * often and the byte comparison must separate them (a self-test mode). */
   int32_t dedup;
 } ks_params;
 
@@ -174,6 +199,8 @@ typedef struct {
   int32_t* exec_counts; /* [n_items] optional: states item k ran on (with dedup: the
                            distinct ones, the reference included) */
   float* final_states;  /* [C][T][d] optional: every cell's state after the last item */
+  int32_t* dedup_rejected; /* [n_items] optional, distinct-state execution only: the
+                              fingerprint matches item k's byte comparison rejected */
 } ks_result;
 
 /* Library version string (static storage). */
@@ -271,8 +298,13 @@ KS_API ks_status ks_reference_forward(const ks_model_desc* model, const ks_layer
  * that loads the library holds until the process exits.
  *  - The first call on a device looks up that array's device address (with
  *    that device current); make that first call before any stream capture.
- *  - Sizes whose scratch exceeds 8 MiB (T * (d_model + 2 Hq hd + 2 ffn) *
- *    bytes-per-element, plus alignment) are rejected with KS_ERR_UNSUPPORTED.
+ *    The address is then kept for the life of the process, so it belongs to
+ *    the device's primary context: do not call this entry point after a
+ *    cudaDeviceReset of that device, nor with a different context current.
+ *  - Sizes whose scratch exceeds 8 MiB are rejected with KS_ERR_UNSUPPORTED.
+ *    The scratch is T * (d_model + 2 Hq hd + 2 ffn) * bytes-per-element
+ *    (4 for fp32 weights, 2 for bf16) for the operands plus T * head_dim * 4
+ *    bytes for the RoPE table, each of the six pieces rounded up to 256 bytes.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents; every byte a call reads it has written first, so nothing needs
  *    clearing.  Calls that overlap on the GPU (other streams, other threads)

@@ -37,12 +37,17 @@ class ModelDesc(ctypes.Structure):
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down")]
+                ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down", "wk", "wv")]
+
+
+KS_KV_CACHE, KS_KV_WINDOW = 0, 1
+KV_MODES = {"cache": KS_KV_CACHE, "window": KS_KV_WINDOW}
 
 
 class CacheDesc(ctypes.Structure):
     _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
-                ("cache_rows", ctypes.c_int64), ("ctx", ctypes.c_int32)]
+                ("cache_rows", ctypes.c_int64), ("ctx", ctypes.c_int32),
+                ("kv_mode", ctypes.c_int32)]
 
 
 KS_BUDGET_AT_MOST, KS_BUDGET_EXACT = 0, 1
@@ -60,7 +65,7 @@ class Result(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("status", "values", "sets", "used_w", "t_draft", "bp", "cos_skip",
                  "cos_exec", "tpt", "best", "best_tpt", "ref_states", "exec_counts",
-                 "final_states")]
+                 "final_states", "dedup_rejected")]
 
 
 class KernelStat(ctypes.Structure):
@@ -174,31 +179,43 @@ def model_desc(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, ffn, rms_eps,
 
 def _layer_shapes(m: ModelDesc) -> Dict[str, tuple]:
     d, qd, F = m.d_model, m.n_q_heads * m.head_dim, m.ffn
+    kvd = m.n_kv_heads * m.head_dim
     return {"attn_norm": (d,), "wq": (qd, d), "wo": (d, qd), "mlp_norm": (d,),
-            "w_gate": (F, d), "w_up": (F, d), "w_down": (d, F)}
+            "w_gate": (F, d), "w_up": (F, d), "w_down": (d, F), "wk": (kvd, d), "wv": (kvd, d)}
+
+
+OPTIONAL_WEIGHTS = ("wk", "wv")        # read only by the window key/value reading
 
 
 def layer_array(layers: Sequence[Dict[str, torch.Tensor]], wdtype: torch.dtype,
                 model: Optional[ModelDesc] = None):
     """Host array of the layers' device weight pointers; with a model, the
-    layer count and every weight's shape are checked against it."""
+    layer count and every weight's shape are checked against it.  wk / wv are
+    optional (NULL when a layer has none)."""
     if model is not None and len(layers) != model.n_layers:
         raise KnapSpecError(f"model has {model.n_layers} layers, got {len(layers)}")
     if model is not None:
         for i, L in enumerate(layers):
             for name, shape in _layer_shapes(model).items():
+                if name in OPTIONAL_WEIGHTS and L.get(name) is None:
+                    continue
                 _shape(L[name], shape, f"layers[{i}].{name}")
     arr = (LayerWeights * len(layers))()
     for i, L in enumerate(layers):
-        for name in ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down"):
+        for name in ("attn_norm", "wq", "wo", "mlp_norm", "w_gate", "w_up", "w_down", "wk", "wv"):
+            if name in OPTIONAL_WEIGHTS and L.get(name) is None:
+                continue
             setattr(arr[i], name, _dev(L[name], wdtype, f"layers[{i}].{name}"))
     return arr
 
 
 def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int,
-               model: Optional[ModelDesc] = None) -> CacheDesc:
+               model: Optional[ModelDesc] = None, kv: str = "cache") -> CacheDesc:
     """The KV cache [L][rows][Hkv][hd] of K and V; with a model, L >= n_layers,
-    Hkv, hd and the dtype are checked against it."""
+    Hkv, hd and the dtype are checked against it.  kv: "cache" (every key and
+    value from the cache) or "window" (the window's recomputed from each state)."""
+    if kv not in KV_MODES:
+        raise KnapSpecError(f"kv must be one of {sorted(KV_MODES)}, got {kv!r}")
     if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
         raise KnapSpecError("k_cache / v_cache must both be [L][rows][Hkv][hd]")
     dt = None
@@ -209,17 +226,20 @@ def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int,
                                 f"[{model.n_kv_heads}][{model.head_dim}], got {tuple(k_cache.shape)}")
         dt = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
     return CacheDesc(_dev(k_cache, dt, "k_cache"), _dev(v_cache, dt, "v_cache"),
-                     k_cache.shape[1], ctx)
+                     k_cache.shape[1], ctx, KV_MODES[kv])
 
 
 def params(gamma_max: int, n_bins: int = 0, alpha_lo: float = 0.5, alpha_scale: float = 0.5,
            alpha_max: float = 0.99, budget_mode: str = "at_most",
            prune_tau: Optional[float] = None, skip_cap: Optional[int] = None,
-           dedup: bool = False) -> Params:
+           dedup=False) -> Params:
+    """dedup: False / True, or "weak" for 8-bit fingerprints (every fold then
+    rests on the byte comparison; a self-test of that check)."""
     mode = {"at_most": KS_BUDGET_AT_MOST, "exact": KS_BUDGET_EXACT}[budget_mode]
+    dd = 2 if dedup == "weak" else (1 if dedup else 0)
     return Params(gamma_max, n_bins, mode, alpha_lo, alpha_scale, alpha_max,
                   float("-inf") if prune_tau is None else float(prune_tau),
-                  -1 if skip_cap is None else int(skip_cap), 1 if dedup else 0)
+                  -1 if skip_cap is None else int(skip_cap), dd)
 
 
 # ---------------------------------------------------------------- calls
@@ -429,6 +449,7 @@ class SolveOutputs:
     ref_states: Optional[torch.Tensor] = None
     exec_counts: Optional[torch.Tensor] = None
     final_states: Optional[torch.Tensor] = None
+    dedup_rejected: Optional[torch.Tensor] = None
 
 
 class Solver:
@@ -438,13 +459,14 @@ class Solver:
                  k_cache: torch.Tensor, v_cache: torch.Tensor, ctx: int, T: int,
                  t: Sequence[float], prm: Params, w: Optional[Sequence[int]] = None,
                  keep_bp: bool = True, keep_cos: bool = False, keep_tpt: bool = True,
-                 keep_ref: bool = True, keep_final: bool = False, device="cuda"):
+                 keep_ref: bool = True, keep_final: bool = False, device="cuda",
+                 kv: str = "cache"):
         self.model = model
         self.wdtype = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
         self._layers_keep = layers
         self.layers = layer_array(layers, self.wdtype, model)
         self._cache_keep = (k_cache, v_cache)
-        self.cache = cache_desc(k_cache, v_cache, ctx, model)
+        self.cache = cache_desc(k_cache, v_cache, ctx, model, kv=kv)
         self.T = T
         self.t = list(map(float, t))
         self.prm = prm
@@ -468,13 +490,14 @@ class Solver:
             tpt=z(C, prm.gamma_max, dt=torch.float64) if keep_tpt else None,
             ref_states=z(n + 1, T, model.d_model, dt=torch.float32) if keep_ref else None,
             exec_counts=z(n, dt=torch.int32),
-            final_states=z(C, T, model.d_model, dt=torch.float32) if keep_final else None)
+            final_states=z(C, T, model.d_model, dt=torch.float32) if keep_final else None,
+            dedup_rejected=z(n, dt=torch.int32) if prm.dedup else None)
         o = self.out
         p = lambda x: None if x is None else x.data_ptr()
         self.result = Result(p(o.status), p(o.values), p(o.sets), p(o.used_w), p(o.t_draft),
                              p(o.bp), p(o.cos_skip), p(o.cos_exec), p(o.tpt), p(o.best),
                              p(o.best_tpt), p(o.ref_states), p(o.exec_counts),
-                             p(o.final_states))
+                             p(o.final_states), p(o.dedup_rejected))
         self._t_arr = (ctypes.c_double * n)(*self.t)
         self._w_arr = (ctypes.c_int32 * n)(*self.w)
 

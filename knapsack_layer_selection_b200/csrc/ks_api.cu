@@ -63,6 +63,11 @@ static ks_status check_cache(const ks_model_desc* m, const ks_cache_desc* c, int
   if (!c || !c->k_cache || !c->v_cache) return fail(KS_ERR_INVALID_ARG, "cache is NULL");
   KS_TRY(check_aligned16({c->k_cache, c->v_cache}, "cache"));
   if (c->ctx < 0) return fail(KS_ERR_INVALID_ARG, "ctx must be >= 0");
+  if (c->kv_mode != KS_KV_CACHE && c->kv_mode != KS_KV_WINDOW)
+    return fail(KS_ERR_INVALID_ARG, "cache kv_mode must be KS_KV_CACHE or KS_KV_WINDOW");
+  if (c->kv_mode == KS_KV_WINDOW && m->wdtype == KS_BF16 && 128 % T)
+    return fail(KS_ERR_UNSUPPORTED,
+                "KS_KV_WINDOW with bf16 weights needs T to divide 128 (whole states per row tile)");
   if (c->cache_rows < (int64_t)c->ctx + T)
     return fail(KS_ERR_INVALID_ARG, "cache_rows must be >= ctx + T");
   // fp32 weights run the SIMT attention, which keeps a row's scores in shared memory
@@ -71,14 +76,22 @@ static ks_status check_cache(const ks_model_desc* m, const ks_cache_desc* c, int
   return KS_OK;
 }
 
-static ks_status check_layers(const ks_model_desc* m, const ks_layer_weights* layers) {
+static ks_status check_layers(const ks_model_desc* m, const ks_layer_weights* layers,
+                              const ks_cache_desc* c) {
   if (!layers) return fail(KS_ERR_INVALID_ARG, "layers is NULL");
+  const bool window = c && c->kv_mode == KS_KV_WINDOW;
   for (int l = 0; l < m->n_layers; ++l) {
     const ks_layer_weights& L = layers[l];
     if (!L.attn_norm || !L.wq || !L.wo || !L.mlp_norm || !L.w_gate || !L.w_up || !L.w_down)
       return fail(KS_ERR_INVALID_ARG, "layer " + std::to_string(l) + " has a NULL weight");
     KS_TRY(check_aligned16({L.attn_norm, L.wq, L.wo, L.mlp_norm, L.w_gate, L.w_up, L.w_down},
                            "layer weights"));
+    if (window) {
+      if (!L.wk || !L.wv)
+        return fail(KS_ERR_INVALID_ARG,
+                    "layer " + std::to_string(l) + ": KS_KV_WINDOW needs wk and wv");
+      KS_TRY(check_aligned16({L.wk, L.wv}, "layer weights"));
+    }
   }
   return KS_OK;
 }
@@ -90,6 +103,7 @@ struct Workspace {
   void *xh;                   // [C+1][T][d] act: the current item's normalised operand
   void *q, *att;              // [(C+1)T][qd] act
   void *gb, *ub;              // [(C+1)T][ffn] act
+  void *kw, *vw;              // [(C+1)T][Hkv*hd] act: window keys / values (KS_KV_WINDOW)
   uint8_t* bp;                // [n_items][C]
   uint8_t *valid_a, *valid_b; // [C] exact-budget validity, ping-pong
   uint64_t *hash_a, *hash_b;  // [C+1] state fingerprints (distinct-state execution), ping-pong
@@ -128,6 +142,9 @@ static Workspace carve(const ks_model_desc* m, long long n_slots, long long T, c
   w.att = take(R * qd * ab);
   w.gb = take(R * F * ab);
   w.ub = take(R * F * ab);
+  const long long kvd = (long long)m->n_kv_heads * m->head_dim;
+  w.kw = take(R * kvd * ab);
+  w.vw = take(R * kvd * ab);
   w.bp = (uint8_t*)take(n_items * C);
   w.valid_a = (uint8_t*)take(C);
   w.valid_b = (uint8_t*)take(C);
@@ -198,19 +215,48 @@ static ks_status sublayer(const Ctx& c, int k, const float* in, int E, float* ou
                                    c.st));
       }
     }
+    const bool window = c.cache->kv_mode == KS_KV_WINDOW;
+    const void* kw = nullptr;
+    const void* vw = nullptr;
+    if (window) {
+      // the window positions' keys and values from the candidates' own normalised
+      // state: k = RoPE(x^ Wk^T) at position ctx + t (the query's rotation), v = x^ Wv^T
+      const int kvd = m->n_kv_heads * m->head_dim;
+      ProfScope ps(KK_GEMM_KV, c.st, 2.0 * 2.0 * Rd * kvd * d,
+                   (Rd * d + 2.0 * kvd * d) * ab + 2.0 * Rd * kvd * ab, tc ? 2 : 3);
+      if (tc) {
+        KS_TRY(tc_gemm(xh, L.wk, nullptr, c.ws.kw, nullptr, R, kvd, d, EPI_ROPE_BF16, c.ws.rope,
+                       c.T, m->head_dim, c.status, c.st, dyn_cells));
+        KS_TRY(tc_gemm(xh, L.wv, nullptr, c.ws.vw, nullptr, R, kvd, d, EPI_STORE_BF16, nullptr,
+                       c.T, m->head_dim, c.status, c.st, dyn_cells));
+      } else {
+        KS_TRY(launch_gemm_simt(xh, c.act, L.wk, m->wdtype, c.ws.kw, false, nullptr, R, kvd, d,
+                                c.st));
+        KS_TRY(launch_rope_inplace(c.ws.kw, c.act, c.ws.rope, R, m->n_kv_heads, m->head_dim, c.T,
+                                   c.st));
+        KS_TRY(launch_gemm_simt(xh, c.act, L.wv, m->wdtype, c.ws.vw, false, nullptr, R, kvd, d,
+                                c.st));
+      }
+      kw = c.ws.kw;
+      vw = c.ws.vw;
+    }
     {
       const double T = c.T, ctx = c.cache->ctx;
       const double keys = (double)E * (T * ctx + T * (T + 1) / 2);   // sum over rows of visible keys
-      const double kv_bytes = 2.0 * (ctx + T) * m->n_kv_heads * m->head_dim * wb;
+      // cache keys/values read: ctx + T rows, or ctx rows plus the window tensors
+      const double kv_bytes = window ? 2.0 * ctx * m->n_kv_heads * m->head_dim * wb +
+                                           2.0 * Rd * m->n_kv_heads * m->head_dim * ab
+                                     : 2.0 * (ctx + T) * m->n_kv_heads * m->head_dim * wb;
       ProfScope ps(KK_ATTN, c.st, 4.0 * m->n_q_heads * m->head_dim * keys,
                    2.0 * Rd * qd * ab + kv_bytes);
       if (tc) {
         KS_TRY(tc_attention(c.ws.q, kc, vc, c.cache->cache_rows, R, c.T, m->n_q_heads,
                             m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.status, c.st,
-                            dyn_cells));
+                            dyn_cells, kw, vw));
       } else {
         KS_TRY(launch_attention_simt(c.ws.q, c.act, kc, vc, m->wdtype, R, c.T, m->n_q_heads,
-                                     m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.st));
+                                     m->n_kv_heads, m->head_dim, c.cache->ctx, c.ws.att, c.st,
+                                     kw, vw));
       }
     }
     {
@@ -370,7 +416,7 @@ static ks_status make_ctx(const ks_model_desc* model, const ks_layer_weights* la
   KS_TRY(check_model(model));
   KS_TRY(check_T(T));
   KS_TRY(check_cache(model, cache, T));
-  KS_TRY(check_layers(model, layers));
+  KS_TRY(check_layers(model, layers, cache));
   if (!workspace) return fail(KS_ERR_INVALID_ARG, "workspace is NULL");
   if ((uintptr_t)workspace % 256) return fail(KS_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   const size_t need = carve(model, n_cells, T, nullptr).total;
@@ -491,6 +537,8 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     return fail(KS_ERR_INVALID_ARG, "solve: budget_mode must be KS_BUDGET_AT_MOST or KS_BUDGET_EXACT");
   if (params->prune_tau != params->prune_tau)
     return fail(KS_ERR_INVALID_ARG, "solve: prune_tau is NaN (use -INFINITY to turn it off)");
+  if (params->dedup < 0 || params->dedup > 2)
+    return fail(KS_ERR_INVALID_ARG, "solve: dedup must be 0 (off), 1 (on) or 2 (8-bit fingerprints)");
   KS_TRY(check_aligned16({x0, ref, out->ref_states, out->final_states}, "solve"));
   const int n_items = 2 * model->n_layers;
   std::vector<int32_t> ww;
@@ -514,6 +562,14 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
   const long long cell = (long long)T * model->d_model;
 
   KS_CUDA_TRY(cudaMemsetAsync(out->status, 0, sizeof(int32_t), st));
+  if (cache->kv_mode == KS_KV_WINDOW && params->dedup) {
+    // rows past a compacted batch's live count are read (and masked) by the
+    // attention's window block: they must hold finite values from the start
+    const size_t kvb = (size_t)(C + 1) * T * model->n_kv_heads * model->head_dim *
+                       act_bytes(c.act);
+    KS_CUDA_TRY(cudaMemsetAsync(c.ws.kw, 0, kvb, st));
+    KS_CUDA_TRY(cudaMemsetAsync(c.ws.vw, 0, kvb, st));
+  }
   {
     ProfScope ps(KK_ROPE_TABLE, st, 0.0, 0.0);
     KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, st));
@@ -554,7 +610,14 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
       {
         ProfScope ps(KK_DEDUP, st, 0.0, (E + 1.0) * 9.0);
         KS_TRY(launch_dedup(hprev, vprev, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
-                            out->exec_counts ? out->exec_counts + k : nullptr, st));
+                            out->exec_counts ? out->exec_counts + k : nullptr,
+                            params->dedup == 2, st));
+      }
+      {
+        ProfScope ps(KK_DEDUP_VERIFY, st, 0.0, 2.0 * (E + 1.0) * cell * 4.0);
+        KS_TRY(launch_dedup_verify(prev, cell, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
+                                   out->exec_counts ? out->exec_counts + k : nullptr,
+                                   out->dedup_rejected ? out->dedup_rejected + k : nullptr, st));
       }
       {
         ProfScope ps(KK_GATHER, st, 0.0, 2.0 * (E + 1.0) * cell * (4.0 + xb));
@@ -641,9 +704,12 @@ ks_status ks_reference_forward_noalloc(const ks_model_desc* model,
   KS_TRY(check_model(model));
   KS_TRY(check_T(T));
   KS_TRY(check_cache(model, cache, T));
-  KS_TRY(check_layers(model, layers));
+  KS_TRY(check_layers(model, layers, cache));
   if (!x0 || !ref_out) return fail(KS_ERR_INVALID_ARG, "x0 / ref_out is NULL");
   KS_TRY(check_aligned16({x0, ref_out}, "reference_forward_noalloc"));
+  if (cache->kv_mode != KS_KV_CACHE)
+    return fail(KS_ERR_UNSUPPORTED,
+                "reference_forward_noalloc: only KS_KV_CACHE (use ks_reference_forward)");
   Workspace w;
   const size_t need = carve_sublayer_only(model, T, nullptr, &w);
   if (need > kStaticScratchBytes)

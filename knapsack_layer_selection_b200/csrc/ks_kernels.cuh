@@ -33,10 +33,14 @@ ks_status launch_swiglu_inplace(void* g, const void* u, int act, long long n, cu
 
 // o[r][h] = softmax(q[r][h] . K[0..ctx+t]^T / sqrt(hd)) . V  with t = r % T and kv head
 // h / (Hq / Hkv).  q, o: [R][Hq][hd] activation dtype; kc, vc: one layer's cache
-// [rows][Hkv][hd] in the weight dtype.  CUDA-core version.
+// [rows][Hkv][hd] in the weight dtype.  With kw, vw ([R][Hkv][hd], activation
+// dtype) the positions ctx + j, j = 0 .. t, take key / value row (r - t + j) of
+// kw / vw -- the window of row r's own state -- instead of the cache.
+// CUDA-core version.
 ks_status launch_attention_simt(const void* q, int act, const void* kc, const void* vc, int wdt,
                                 int R, int T, int Hq, int Hkv, int hd, int ctx, void* o,
-                                cudaStream_t st);
+                                cudaStream_t st, const void* kw = nullptr,
+                                const void* vw = nullptr);
 
 // dst[c] = src for c in [0, n_copies), each copy n_elems floats.
 ks_status launch_broadcast(float* dst, const float* src, int n_copies, long long n_elems,
@@ -65,7 +69,12 @@ ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float e
 
 // Distinct-state compaction of the next execute batch (slots 0..n-1): see ks_select.cu.
 ks_status launch_dedup(const uint64_t* hash, const uint8_t* valid, int n, int* map, int* uniq,
-                       int* count, int32_t* count_out, cudaStream_t st);
+                       int* count, int32_t* count_out, bool weak, cudaStream_t st);
+// Byte comparison of every fold launch_dedup made; a slot whose state differs
+// from its representative's gets its own compacted entry.
+ks_status launch_dedup_verify(const float* states, long long cell, int n, int* map, int* uniq,
+                              int* count, int32_t* count_out, int32_t* rejected_out,
+                              cudaStream_t st);
 ks_status launch_gather(const int* uniq, const int* count, int max_count, long long cell,
                         const float* states, const void* xh, int act, float* states_c, void* xh_c,
                         cudaStream_t st);

@@ -49,7 +49,7 @@ const char* kernel_kind_name(int k) {
                                         "gemm_gateup_swiglu", "gemm_down_residual", "rope",
                                         "swiglu", "attention", "select_bp", "reconstruct",
                                         "tpt_argmax", "init_states", "rope_table", "dedup",
-                                        "gather"};
+                                        "gather", "dedup_verify", "gemm_kv_window"};
   return (k >= 0 && k < KK_COUNT) ? names[k] : "?";
 }
 

@@ -23,6 +23,8 @@ enum KernelKind {
   KK_ROPE_TABLE,
   KK_DEDUP,
   KK_GATHER,
+  KK_DEDUP_VERIFY,
+  KK_GEMM_KV,
   KK_COUNT
 };
 

@@ -405,21 +405,24 @@ ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float e
 
 // ---------------------------------------------------------------- distinct-state compaction
 // Slots 0..n-1 of the state buffer (slot 0 = reference, slot s = cell s-1) are
-// the next item's execute sources.  Slots holding bit-identical states (equal
-// fingerprints) and valid are folded onto their first occurrence: map[s] is the
-// compacted index of slot s's state (-1 for an invalid cell), uniq[u] the slot
-// of the u-th distinct state, *count the number of distinct states.  One CTA.
+// the next item's execute sources.  Valid slots with equal fingerprints are
+// folded onto their first occurrence: map[s] is the compacted index of slot
+// s's state (-1 for an invalid cell), uniq[u] the slot of the u-th distinct
+// state, *count the number of distinct states.  One CTA.  A fold is only a
+// candidate until dedup_verify_kernel has compared the two states' bytes.
+// With `weak`, only the fingerprints' low 8 bits are compared (self-test mode).
 constexpr int kDedupThreads = 1024;
 constexpr int kDedupMax = 3072;
 
 __global__ void __launch_bounds__(kDedupThreads) dedup_kernel(
     const uint64_t* __restrict__ hash, const uint8_t* __restrict__ valid, int n,
     int* __restrict__ map, int* __restrict__ uniq, int* __restrict__ count,
-    int32_t* __restrict__ count_out) {
+    int32_t* __restrict__ count_out, int weak) {
   __shared__ uint64_t h[kDedupMax];
   __shared__ int first[kDedupMax];
   __shared__ int scan[kDedupThreads];
-  for (int s = threadIdx.x; s < n; s += blockDim.x) h[s] = hash[s];
+  const uint64_t keep = weak ? 0xffull : ~0ull;
+  for (int s = threadIdx.x; s < n; s += blockDim.x) h[s] = hash[s] & keep;
   __syncthreads();
   for (int s = threadIdx.x; s < n; s += blockDim.x) {
     const bool ok = s == 0 || !valid || valid[s - 1];
@@ -469,9 +472,55 @@ __global__ void __launch_bounds__(kDedupThreads) dedup_kernel(
 }
 
 ks_status launch_dedup(const uint64_t* hash, const uint8_t* valid, int n, int* map, int* uniq,
-                       int* count, int32_t* count_out, cudaStream_t st) {
+                       int* count, int32_t* count_out, bool weak, cudaStream_t st) {
   if (n > kDedupMax) return fail(KS_ERR_UNSUPPORTED, "dedup: more than 3071 budget cells");
-  dedup_kernel<<<1, kDedupThreads, 0, st>>>(hash, valid, n, map, uniq, count, count_out);
+  dedup_kernel<<<1, kDedupThreads, 0, st>>>(hash, valid, n, map, uniq, count, count_out,
+                                            weak ? 1 : 0);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+// Block s (one per slot) compares slot s's state with the slot it was folded
+// onto, word by word as bit patterns.  On any difference the slot gets its own
+// compacted entry, appended after the distinct states found so far (count is
+// raised atomically; the entries' order does not matter because every row of
+// the batch is computed independently of its position).  Only block s writes
+// map[s], and uniq entries below the dedup kernel's count are never rewritten.
+constexpr int kVerifyThreads = 256;
+
+__global__ void __launch_bounds__(kVerifyThreads) dedup_verify_kernel(
+    const uint4* __restrict__ states, long long cell4, int* __restrict__ map,
+    int* __restrict__ uniq, int* __restrict__ count, int32_t* __restrict__ count_out,
+    int32_t* __restrict__ rejected_out) {
+  const int s = blockIdx.x;
+  const int u = map[s];
+  if (u < 0) return;
+  const int r = uniq[u];
+  if (r == s) return;               // u, r are the same for the whole block
+  const uint4* a = states + (long long)s * cell4;
+  const uint4* b = states + (long long)r * cell4;
+  int d = 0;
+  for (long long i = threadIdx.x; i < cell4; i += blockDim.x) {
+    const uint4 x = a[i], y = b[i];
+    d |= (x.x != y.x) | (x.y != y.y) | (x.z != y.z) | (x.w != y.w);
+  }
+  if (__syncthreads_or(d) && threadIdx.x == 0) {
+    const int j = atomicAdd(count, 1);
+    uniq[j] = s;
+    map[s] = j;
+    if (count_out) atomicAdd(count_out, 1);
+    if (rejected_out) atomicAdd(rejected_out, 1);
+  }
+}
+
+ks_status launch_dedup_verify(const float* states, long long cell, int n, int* map, int* uniq,
+                              int* count, int32_t* count_out, int32_t* rejected_out,
+                              cudaStream_t st) {
+  if (cell % 4) return fail(KS_ERR_UNSUPPORTED, "dedup: T*d must be a multiple of 4");
+  if (n <= 0) return KS_OK;
+  if (rejected_out) KS_CUDA_TRY(cudaMemsetAsync(rejected_out, 0, sizeof(int32_t), st));
+  dedup_verify_kernel<<<n, kVerifyThreads, 0, st>>>((const uint4*)states, cell / 4, map, uniq,
+                                                   count, count_out, rejected_out);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }

@@ -208,7 +208,9 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(const TQ* __restric
                                                              const TKV* __restrict__ vc,
                                                              TQ* __restrict__ o, int T, int Hq,
                                                              int Hkv, int hd, int ctx,
-                                                             float scale) {
+                                                             float scale,
+                                                             const TQ* __restrict__ kw,
+                                                             const TQ* __restrict__ vw) {
   extern __shared__ float sm[];
   float* qs = sm;             // [hd]
   float* sc = sm + hd;        // [ctx + T]
@@ -222,11 +224,19 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(const TQ* __restric
   const TQ* qp = q + (r * Hq + h) * hd;
   for (int i = threadIdx.x; i < hd; i += blockDim.x) qs[i] = Elem<TQ>::to_f(qp[i]);
   __syncthreads();
+  // window reading: positions ctx + j' (j' <= t) are row (r - t + j') of kw / vw
+  const long long w0 = r - t - ctx;
+  const bool window = kw != nullptr;
   float mx = -INFINITY;
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const TKV* kp = kc + j * kv_row + (long long)g * hd;
     float s = 0.f;
-    for (int i = 0; i < hd; ++i) s = fmaf(qs[i], Elem<TKV>::to_f(kp[i]), s);
+    if (window && j >= ctx) {
+      const TQ* kp = kw + (w0 + j) * kv_row + (long long)g * hd;
+      for (int i = 0; i < hd; ++i) s = fmaf(qs[i], Elem<TQ>::to_f(kp[i]), s);
+    } else {
+      const TKV* kp = kc + j * kv_row + (long long)g * hd;
+      for (int i = 0; i < hd; ++i) s = fmaf(qs[i], Elem<TKV>::to_f(kp[i]), s);
+    }
     s *= scale;
     sc[j] = s;
     mx = fmaxf(mx, s);
@@ -252,15 +262,22 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(const TQ* __restric
   TQ* op = o + (r * Hq + h) * hd;
   for (int i = threadIdx.x; i < hd; i += blockDim.x) {
     const TKV* vp = vc + (long long)g * hd + i;
+    const int nc = window ? ctx : n;             // keys read from the cache
     float acc = 0.f;
-    for (int j = 0; j < n; ++j) acc = fmaf(sc[j], Elem<TKV>::to_f(vp[j * kv_row]), acc);
+    for (int j = 0; j < nc; ++j) acc = fmaf(sc[j], Elem<TKV>::to_f(vp[j * kv_row]), acc);
+    if (window) {
+      const TQ* wp = vw + (long long)g * hd + i;
+      for (int j = ctx; j < n; ++j) acc = fmaf(sc[j], Elem<TQ>::to_f(wp[(w0 + j) * kv_row]), acc);
+    }
     op[i] = Elem<TQ>::from_f(acc * inv);
   }
 }
 
 ks_status launch_attention_simt(const void* q, int act, const void* kc, const void* vc, int wdt,
                                 int R, int T, int Hq, int Hkv, int hd, int ctx, void* o,
-                                cudaStream_t st) {
+                                cudaStream_t st, const void* kw, const void* vw) {
+  if ((kw == nullptr) != (vw == nullptr))
+    return fail(KS_ERR_INVALID_ARG, "attention_simt: window keys and values go together");
   if (R <= 0) return KS_OK;
   const size_t smem = (size_t)(hd + ctx + T) * sizeof(float);
   if (smem > 200 * 1024) return fail(KS_ERR_UNSUPPORTED, "attention_simt: context too long");
@@ -270,13 +287,13 @@ ks_status launch_attention_simt(const void* q, int act, const void* kc, const vo
     auto k = attention_simt_kernel<float, float>;
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     k<<<grid, block, smem, st>>>((const float*)q, (const float*)kc, (const float*)vc, (float*)o,
-                                 T, Hq, Hkv, hd, ctx, scale);
+                                 T, Hq, Hkv, hd, ctx, scale, (const float*)kw, (const float*)vw);
   } else if (act == ACT_BF16 && wdt == KS_BF16) {
     auto k = attention_simt_kernel<__nv_bfloat16, __nv_bfloat16>;
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     k<<<grid, block, smem, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)kc,
                                  (const __nv_bfloat16*)vc, (__nv_bfloat16*)o, T, Hq, Hkv, hd, ctx,
-                                 scale);
+                                 scale, (const __nv_bfloat16*)kw, (const __nv_bfloat16*)vw);
   } else {
     return fail(KS_ERR_UNSUPPORTED, "attention_simt: dtype combination");
   }

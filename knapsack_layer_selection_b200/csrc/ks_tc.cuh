@@ -45,10 +45,13 @@ ks_status make_tmap_2d(CUtensorMap* m, const void* base, long long rows, long lo
 
 // Causal GQA attention on the tensor cores: q, out [R][Hq][hd] bf16 (row r is
 // evaluation token r % T), kc/vc one layer of the cache [cache_rows][Hkv][hd]
-// bf16; token t attends to positions 0 .. ctx + t.  hd = 64 or 128.
+// bf16; token t attends to positions 0 .. ctx + t.  hd = 64 or 128.  With kw,
+// vw ([R][Hkv][hd] bf16, T dividing 128) the window positions ctx .. ctx + t
+// take row r's own state's keys / values (rows r - t .. r) instead of the cache.
 ks_status tc_attention(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
                        int T, int Hq, int Hkv, int hd, int ctx, void* out, int32_t* status,
-                       cudaStream_t st, const int* dyn_cells = nullptr);
+                       cudaStream_t st, const int* dyn_cells = nullptr,
+                       const void* kw = nullptr, const void* vw = nullptr);
 
 int sm_count();
 

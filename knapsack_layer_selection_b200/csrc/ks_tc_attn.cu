@@ -114,6 +114,7 @@ struct AttnParams {
   int R, T, Hq, Hkv, ctx, n_keys, n_blocks;
   float scale_log2;
   const int* dyn_cells;   // optional device count: R = min(R, *dyn_cells * T) at run time
+  int window;             // window reading: the last block holds the tile's own window keys
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -221,7 +222,8 @@ __device__ __forceinline__ void regs_inc() {
 template <int HD>
 __global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p_in) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKw,
+                const __grid_constant__ CUtensorMap tmVw, const AttnParams p_in) {
   using C = Cfg<HD>;
   AttnParams p = p_in;
   if (p.dyn_cells) {
@@ -292,36 +294,49 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (p.window) {
+        prefetch_tmap(&tmKw);
+        prefetch_tmap(&tmVw);
+      }
       const uint32_t qf = smem_u32(&tail->q_full);
       mbar_arrive_expect_tx(qf, C::Q_TILE);
       for (int pn = 0; pn < C::PANELS; ++pn)
         tma_load_2d(sbase + pn * C::Q_PANEL, &tmQ, h * HD + pn * 64, m0, qf);
-      // block m of K (V) goes to ring slot m % KST once the MMA of block m - KST is done
-      auto load_kv = [&](const CUtensorMap* tm, int off, uint64_t* full, uint64_t* empty,
-                         int m, int nst, int slot_bytes) -> bool {
+      // block m of K (V) goes to ring slot m % KST once the MMA of block m - KST is done.
+      // Under the window reading the last block is the tile's own rows of the window
+      // keys / values (whole states: T divides 128 and m0 is a multiple of 128).
+      auto load_kv = [&](const CUtensorMap* tm, const CUtensorMap* tmw, int off, uint64_t* full,
+                         uint64_t* empty, int m, int nst, int slot_bytes) -> bool {
         const int s = m % nst;
         if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(m / nst) & 1u) ^ 1u, abort, p.status))
           return false;
         const uint32_t dst = sbase + off + s * slot_bytes;
         const uint32_t fb = smem_u32(&full[s]);
+        const bool win = p.window && m == J - 1;
+        const CUtensorMap* src = win ? tmw : tm;
+        const int row0 = win ? m0 : m * C::BN;
         mbar_arrive_expect_tx(fb, C::KV_BLOCK);
         for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_2d(dst + pn * C::KV_PANEL, tm, g * HD + pn * 64, m * C::BN, fb);
+          tma_load_2d(dst + pn * C::KV_PANEL, src, g * HD + pn * 64, row0, fb);
         return true;
       };
       // in the order the MMAs consume them: K_0, K_1, then K_{j+2}, V_j for j = 0, 1, ...
       int nk = 0, nv = 0;                       // blocks whose K / V loads were issued
       bool ok = true;
       while (ok && nk < J && nk < 2) {
-        ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST, C::KV_BLOCK);
+        ok = load_kv(&tmK, &tmKw, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST, C::KV_BLOCK);
         if (ok) ++nk;
       }
       while (ok && nv < J) {
         if (nk < J) {
-          if (!(ok = load_kv(&tmK, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST, C::KV_BLOCK))) break;
+          if (!(ok = load_kv(&tmK, &tmKw, C::OFF_K, tail->k_full, tail->k_empty, nk, C::KST,
+                             C::KV_BLOCK)))
+            break;
           ++nk;
         }
-        if (!(ok = load_kv(&tmV, C::OFF_V, tail->v_full, tail->v_empty, nv, C::VST, C::V_SLOT))) break;
+        if (!(ok = load_kv(&tmV, &tmVw, C::OFF_V, tail->v_full, tail->v_empty, nv, C::VST,
+                           C::V_SLOT)))
+          break;
         ++nv;
       }
       // drain the copies still in flight before leaving
@@ -401,6 +416,10 @@ __global__ void __launch_bounds__(384, 1)
     const int row = m0 + r;
     const bool live = row < p.R;
     const int limit = p.ctx + (live ? row % p.T : 0);   // last visible cache position
+    // window reading: context blocks show positions < ctx; the last block shows the
+    // keys lo .. r of the tile (this row's own state, tokens 0 .. t)
+    const int ctx_last = p.ctx - 1;
+    const int win_lo = (r / p.T) * p.T;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t ts = tmem + lane_off + C::TMEM_S + G * C::BN;
     const uint32_t tp = tmem + lane_off + C::TMEM_P;
@@ -437,7 +456,18 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tail->s_free[G]));   // S_{i+2} may be computed now
-      if (i * C::BN + C::BN - 1 > p.ctx) {       // a key of this block may be past the window
+      if (p.window) {
+        if (i == J - 1) {                        // the tile's own window keys
+#pragma unroll
+          for (int e = 0; e < NC; ++e)
+            if (e < win_lo || e > r) sc[e] = -INFINITY;
+        } else if (i * C::BN + C::BN - 1 > ctx_last) {   // a context block reaching past ctx
+          const int key0 = i * C::BN;
+#pragma unroll
+          for (int e = 0; e < NC; ++e)
+            if (key0 + e > ctx_last) sc[e] = -INFINITY;
+        }
+      } else if (i * C::BN + C::BN - 1 > p.ctx) {   // a key of this block may be past the window
         const int key0 = i * C::BN;
 #pragma unroll
         for (int e = 0; e < NC; ++e)
@@ -555,7 +585,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int HD>
 ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int T, int Hq, int Hkv,
                       int ctx, void* out, int32_t* status, cudaStream_t st,
-                      const int* dyn_cells) {
+                      const int* dyn_cells, const void* kw, const void* vw) {
   using C = Cfg<HD>;
   static std::atomic<unsigned long long> attr{0};
   auto k = attn_kernel<HD>;
@@ -570,11 +600,22 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int 
     KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     return KS_OK;
   }));
-  const int n_keys = ctx + T;
-  CUtensorMap tq, tk, tv;
+  const bool window = kw != nullptr;
+  // keys read from the cache: all ctx + T positions, or the ctx context positions
+  // when the window comes from kw / vw (at least one row, so the map is valid)
+  const int n_keys = window ? ctx : ctx + T;
+  const long long kvd = (long long)Hkv * HD;
+  CUtensorMap tq, tk, tv, tkw, tvw;
   KS_TRY(make_tmap_2d(&tq, q, R, (long long)Hq * HD, (long long)Hq * HD, 64, C::BM));
-  KS_TRY(make_tmap_2d(&tk, kc, n_keys, (long long)Hkv * HD, (long long)Hkv * HD, 64, C::BN));
-  KS_TRY(make_tmap_2d(&tv, vc, n_keys, (long long)Hkv * HD, (long long)Hkv * HD, 64, C::BN));
+  KS_TRY(make_tmap_2d(&tk, kc, n_keys > 0 ? n_keys : 1, kvd, kvd, 64, C::BN));
+  KS_TRY(make_tmap_2d(&tv, vc, n_keys > 0 ? n_keys : 1, kvd, kvd, 64, C::BN));
+  if (window) {
+    KS_TRY(make_tmap_2d(&tkw, kw, R, kvd, kvd, 64, C::BN));
+    KS_TRY(make_tmap_2d(&tvw, vw, R, kvd, kvd, 64, C::BN));
+  } else {
+    tkw = tk;
+    tvw = tv;
+  }
   AttnParams ap;
   ap.out = out;
   ap.status = status;
@@ -584,11 +625,12 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int 
   ap.Hkv = Hkv;
   ap.ctx = ctx;
   ap.n_keys = n_keys;
-  ap.n_blocks = (n_keys + C::BN - 1) / C::BN;
+  ap.n_blocks = (n_keys + C::BN - 1) / C::BN + (window ? 1 : 0);
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)HD));
   ap.dyn_cells = dyn_cells;
+  ap.window = window ? 1 : 0;
   const dim3 grid((R + C::BM - 1) / C::BM, Hq);
-  k<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, ap);
+  k<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, tkw, tvw, ap);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -597,14 +639,18 @@ ks_status launch_attn(const void* q, const void* kc, const void* vc, int R, int 
 
 ks_status tc_attention(const void* q, const void* kc, const void* vc, long long cache_rows, int R,
                        int T, int Hq, int Hkv, int hd, int ctx, void* out, int32_t* status,
-                       cudaStream_t st, const int* dyn_cells) {
+                       cudaStream_t st, const int* dyn_cells, const void* kw, const void* vw) {
   if (R <= 0) return KS_OK;
   if (Hq % Hkv) return fail(KS_ERR_INVALID_ARG, "attention: Hq must be a multiple of Hkv");
   if (cache_rows < (long long)ctx + T) return fail(KS_ERR_INVALID_ARG, "attention: cache too short");
+  if ((kw == nullptr) != (vw == nullptr))
+    return fail(KS_ERR_INVALID_ARG, "attention: window keys and values go together");
+  if (kw && (T < 1 || 128 % T))
+    return fail(KS_ERR_UNSUPPORTED, "attention: the window reading needs T to divide 128");
   if (hd == 128)
-    return launch_attn<128>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
+    return launch_attn<128>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells, kw, vw);
   if (hd == 64)
-    return launch_attn<64>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells);
+    return launch_attn<64>(q, kc, vc, R, T, Hq, Hkv, ctx, out, status, st, dyn_cells, kw, vw);
   return fail(KS_ERR_UNSUPPORTED, "attention: head_dim must be 64 or 128");
 }
 

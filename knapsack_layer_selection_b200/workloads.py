@@ -21,11 +21,16 @@ the paper uses are not available, so every tensor here is drawn at random:
 
 Draw order (one ``torch.Generator`` seeded with ``seed`` on ``device``): for each
 layer in order Wq, Wo, W_gate, W_up, W_down; then the K cache, the V cache, then
-x0.  Each tensor is drawn in fp32 and then rounded to the storage dtype.
+x0.  Each tensor is drawn in fp32 and then rounded to the storage dtype.  Every
+workload that fits in host memory is drawn on the CPU generator (the 64 GB
+Qwen3-32B shape alone is drawn on the GPU's), so that a machine without a GPU
+can reproduce the inputs exactly; ``input_digest`` fingerprints a draw so that
+two machines can confirm they hold the same values.
 """
 from __future__ import annotations
 
 import dataclasses
+import hashlib
 import math
 from typing import Dict, List, Optional, Sequence
 
@@ -104,12 +109,12 @@ WORKLOADS: Dict[str, Workload] = {
     "llama3_8b_8k": Workload("llama3_8b_8k", n_layers=32, d_model=4096, n_q_heads=32,
                              n_kv_heads=8, head_dim=128, ffn=14336, rms_eps=1e-6,
                              rope_base=5e5, ctx=8192, T=16, wdtype="bf16", n_bins=512,
-                             gamma_max=10, gen_device="cuda"),
+                             gamma_max=10, gen_device="cpu"),
     # Llama-3-8B shape, long context, re-solved at 4k / 16k / 32k.
     "llama3_8b_32k": Workload("llama3_8b_32k", n_layers=32, d_model=4096, n_q_heads=32,
                               n_kv_heads=8, head_dim=128, ffn=14336, rms_eps=1e-6,
                               rope_base=5e5, ctx=32768, T=16, wdtype="bf16", n_bins=1024,
-                              gamma_max=10, gen_device="cuda",
+                              gamma_max=10, gen_device="cpu",
                               contexts=(4096, 16384, 32768)),
     # Qwen3-32B shape at 16k context (q-dim 8192 differs from d_model 5120).
     "qwen3_32b_16k": Workload("qwen3_32b_16k", n_layers=64, d_model=5120, n_q_heads=64,
@@ -190,6 +195,22 @@ def make_inputs(wl: Workload, seed: int = 0, device: Optional[str] = None) -> In
     return Inputs(wl, layers, k_cache, v_cache, x0)
 
 
+def window_weights(wl: Workload, seed: int = 2, device: Optional[str] = None
+                   ) -> List[Dict[str, torch.Tensor]]:
+    """Per layer the key/value projections Wk, Wv [Hkv*hd][d] ~ N(0, 0.02^2) in the
+    workload's weight dtype, from their own generator and seed (drawn in layer
+    order, Wk then Wv), so the main draw order above is unchanged.  Only the
+    attention reading that recomputes the window's keys/values uses them."""
+    dev = device or wl.gen_device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dt = torch_dtype(wl)
+    kvd = wl.n_kv_heads * wl.head_dim
+    return [{"wk": _randn((kvd, wl.d_model), LINEAR_STD, dt, gen, dev),
+             "wv": _randn((kvd, wl.d_model), LINEAR_STD, dt, gen, dev)}
+            for _ in range(wl.n_layers)]
+
+
 def truncated(wl: Workload, n_layers: int, ctx: Optional[int] = None) -> Workload:
     """The same workload shape with fewer layers (and optionally another context)."""
     return dataclasses.replace(wl, n_layers=n_layers, ctx=wl.ctx if ctx is None else ctx)
@@ -217,3 +238,26 @@ def random_states(shape: Sequence[int], seed: int, device: str = "cpu",
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32).to(dtype)
+
+
+def input_digest(inp: Inputs) -> str:
+    """SHA-256 of every input tensor's bytes, in draw order (weights layer by layer,
+    then the K cache, the V cache and x0).  Two draws hold the same values iff
+    their digests agree (up to hash collisions)."""
+    h = hashlib.sha256()
+
+    def put(t: torch.Tensor):
+        t = t.detach().contiguous().cpu()
+        if t.dtype == torch.bfloat16:
+            t = t.view(torch.int16)
+        h.update(t.numpy().tobytes())
+
+    for layer in inp.layers:
+        for k in ("wq", "wo", "w_gate", "w_up", "w_down", "attn_norm", "mlp_norm"):
+            put(layer[k])
+    for l in range(inp.k_cache.shape[0]):
+        put(inp.k_cache[l])
+    for l in range(inp.v_cache.shape[0]):
+        put(inp.v_cache[l])
+    put(inp.x0)
+    return h.hexdigest()

@@ -253,3 +253,54 @@ def test_misaligned_device_pointers_are_refused_before_any_launch(lib):
     st = lib.ks_solve(ctypes.byref(m), None, None, 4, q, None, None, t, ctypes.byref(prm), None, 0,
                       ctypes.byref(res), None)
     assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
+
+
+def test_window_reading_and_dedup_mode_are_checked_before_any_launch(lib):
+    """The key/value reading of the cache descriptor, the window reading's Wk / Wv
+    and row-tile condition, and the distinct-state mode are refused on the host."""
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    layers = (B.LayerWeights * 1)()
+    for f, _ in B.LayerWeights._fields_:
+        setattr(layers[0], f, 256)
+    p = ctypes.c_void_p(256)
+    bad_mode = B.CacheDesc(256, 256, 16, 8, 5)
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(bad_mode), 4, 0, p, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 1 and b"kv_mode" in lib.ks_last_error()
+    window = B.CacheDesc(256, 256, 16, 8, B.KS_KV_WINDOW)
+    layers[0].wk = None
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(window), 4, 0, p, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 1 and b"wk and wv" in lib.ks_last_error()
+    layers[0].wk = 256 + 4
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(window), 4, 0, p, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 1 and b"16-byte aligned" in lib.ks_last_error()
+    # without the window reading a layer needs no Wk / Wv
+    layers[0].wk = None
+    layers[0].wv = None
+    cache = B.CacheDesc(256, 256, 16, 8, B.KS_KV_CACHE)
+    st = lib.ks_sublayer_forward(ctypes.byref(m), layers, ctypes.byref(cache), 4, 0, None, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 1 and b"states" in lib.ks_last_error()      # got past the layer checks
+    # bf16 (tensor cores): whole states per 128-row tile
+    mb = B.model_desc(1, 256, 4, 1, 64, 256, 1e-6, 1e4, "bf16")
+    layers[0].wk = 256
+    layers[0].wv = 256
+    w6 = B.CacheDesc(256, 256, 16, 8, B.KS_KV_WINDOW)
+    st = lib.ks_sublayer_forward(ctypes.byref(mb), layers, ctypes.byref(w6), 6, 0, p, 1, p,
+                                 p, 1 << 40, None)
+    assert st == 2 and b"divide 128" in lib.ks_last_error()
+    # the fixed-scratch forward keeps to the cache reading
+    st = lib.ks_reference_forward_noalloc(ctypes.byref(m), layers, ctypes.byref(window), 4, p, p,
+                                          None)
+    assert st == 2 and b"KS_KV_CACHE" in lib.ks_last_error()
+    # distinct-state execution: 0, 1 or 2
+    prm = B.params(4, 8)
+    prm.dedup = 3
+    t = (ctypes.c_double * 2)(1.0, 1.0)
+    res = B.Result(*([256] * 15))
+    st = lib.ks_solve(ctypes.byref(m), None, None, 4, p, None, None, t, ctypes.byref(prm), None, 0,
+                      ctypes.byref(res), None)
+    assert st == 1 and b"dedup must be" in lib.ks_last_error()
+    assert B.params(4, 8, dedup="weak").dedup == 2 and B.params(4, 8, dedup=True).dedup == 1

@@ -144,3 +144,25 @@ def test_set_masks_round_trip_across_words():
             for k in range(n):
                 assert ((int(rows[r][k >> 6]) >> (k & 63)) & 1) == (k in items)
         assert B.sets_to_lists(torch.from_numpy(rows.view(np.int64)), n) == lists
+
+
+def test_window_weights_and_kv_reading():
+    """Wk / Wv are optional weights whose shapes are checked when given; the
+    cache descriptor's key/value reading is one of two names."""
+    wl = W.WORKLOADS["tiny"]
+    m = _model(wl)
+    kvd = wl.n_kv_heads * wl.head_dim
+    inp = W.make_inputs(wl)
+    layers = [dict(L) for L in inp.layers]
+    with pytest.raises(B.KnapSpecError, match=NOT_CUDA):
+        B.layer_array(layers, torch.float32, m)          # no wk / wv: fine up to the pointers
+    layers[1]["wk"] = _t(kvd, wl.d_model)
+    layers[1]["wv"] = _t(kvd + 1, wl.d_model)
+    with pytest.raises(B.KnapSpecError, match=r"layers\[1\]\.wv must have shape"):
+        B.layer_array(layers, torch.float32, m)
+    with pytest.raises(B.KnapSpecError, match="kv must be one of"):
+        B.cache_desc(inp.k_cache, inp.v_cache, wl.ctx, m, kv="recomputed")
+    ww = W.window_weights(wl)
+    assert len(ww) == wl.n_layers and tuple(ww[0]["wk"].shape) == (kvd, wl.d_model)
+    assert torch.equal(ww[0]["wk"], W.window_weights(wl)[0]["wk"])
+    assert abs(ww[0]["wv"].std().item() / 0.02 - 1) < 0.05

@@ -65,3 +65,28 @@ def test_dedup_rejects_grids_beyond_its_table():
         s = B.Solver(m, g.layers, g.k_cache, g.v_cache, wl.ctx, wl.T, t,
                      B.params(wl.gamma_max, 4000, dedup=True))
         s.solve(g.x0)
+
+
+@pytest.mark.parametrize("name,kw", [("small", {}), ("small", {"budget_mode": "exact"}),
+                                     ("tiny", {})])
+def test_byte_check_separates_colliding_fingerprints(name, kw):
+    """With fingerprints cut to 8 bits, unequal states share fingerprints often;
+    every such fold must be rejected by the byte comparison, leaving the result
+    bit-identical to the dense solve."""
+    wl = W.WORKLOADS[name]
+    g = W.make_inputs(wl).to("cuda")
+    s_dense, dense = run(wl, g, **kw)
+    s_weak, weak = run(wl, g, dedup="weak", **kw)
+    s_full, full = run(wl, g, dedup=True, **kw)
+    for k in ("bp", "values", "sets", "used_w", "t_draft", "best", "best_tpt", "ref_states",
+              "cos_skip", "cos_exec"):
+        assert np.array_equal(dense[k], weak[k], equal_nan=True), k
+    rejected_weak = int(s_weak.out.dedup_rejected.sum())
+    rejected_full = int(s_full.out.dedup_rejected.sum())
+    assert rejected_full == 0          # no 64-bit collision expected on these inputs
+    if name == "small":
+        assert rejected_weak > 0       # 8-bit fingerprints: collisions did happen
+    # a rejected fold runs its state on its own, never fewer states than the full check
+    assert np.all(weak["exec_counts"] >= full["exec_counts"])
+    print(f"\n{name} {kw}: 8-bit fingerprints: byte check rejected {rejected_weak} folds; "
+          f"states executed {int(weak['exec_counts'].sum())} (64-bit: {int(full['exec_counts'].sum())})")

@@ -173,3 +173,22 @@ def test_tiny_tpt_and_latency_outputs():
     grid = solver.out.tpt.cpu().numpy()
     b, gm = res["best"]
     assert grid[b, gm - 1] == np.nanmax(grid)
+
+
+@pytest.mark.parametrize("name,mode,dedup", [("tiny", "at_most", True), ("small", "at_most", True),
+                                             ("small", "at_most", "weak"), ("small", "exact", True)])
+def test_distinct_state_solve_matches_oracle(name, mode, dedup):
+    """Distinct-state execution compared with the oracle directly (not only with
+    the dense GPU solve): same rule, same tolerances."""
+    wl, inp, g, solver, res, orc, w, t = solved(name, None, mode)
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    s = B.Solver(m, g.layers, g.k_cache, g.v_cache, wl.ctx, wl.T, t,
+                 B.params(wl.gamma_max, wl.n_bins, budget_mode=mode, dedup=dedup), w=w,
+                 keep_cos=True)
+    s.solve(g.x0)
+    dd = gpu_result(s)
+    rep = compare_solve(orc, dd, w, VAL_TOL[wl.wdtype], wl.n_items, rows_val_gpu=dd["rows"])
+    print(f"\n{name} {mode} dedup={dedup}: executed {int(s.out.exec_counts.sum())} states, "
+          f"byte check rejected {int(s.out.dedup_rejected.sum())} fingerprint matches; {rep}")
+    rep.assert_ok()
