@@ -377,6 +377,33 @@ KS_API ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* la
                    void* workspace, size_t workspace_bytes, ks_result* out, ks_stream_t stream);
 
 /*
+ * The DP re-solved at several contexts in one pass (up to 4).  The review notes
+ * that the layer set is re-optimised every T = 64 / 128 decoding steps while the
+ * context grows ("Assumptions & free parameters") and that Attention latency
+ * grows with the context (Figure 4 caption), so each context has its own item
+ * weights and budget grid, its own reference states and its own attention
+ * window, while the model's weights are the same.  Each item's GEMMs run once
+ * over all contexts' batches, so every weight tile is read once for all of
+ * them; attention and the select run per context.  Context j's results equal
+ * those of ks_solve(model, layers, &caches[j], T, x0[j], NULL, w[j], t[j], ...)
+ * bit for bit (every row's arithmetic is independent of its batch).
+ * caches: HOST [n_ctx] (ctx per context; every kv_mode alike); x0: HOST [n_ctx]
+ * of device [T][d] fp32 pointers; w: HOST [n_ctx] of HOST [n_items] weights (w
+ * or w[j] NULL: quantise t[j] with params->n_bins); t: HOST [n_ctx] of HOST
+ * [n_items] latencies; outs: HOST [n_ctx] results, each sized for its own C.
+ * The workspace must hold ks_workspace_size_contexts(model, n_ctx, C[], T).
+ * Distinct-state execution (params->dedup) is refused with n_ctx > 1.
+ */
+KS_API ks_status ks_workspace_size_contexts(const ks_model_desc* model, int32_t n_ctx,
+                                            const int32_t* n_cells, int32_t T, size_t* bytes);
+KS_API ks_status ks_solve_contexts(const ks_model_desc* model, const ks_layer_weights* layers,
+                                   int32_t n_ctx, const ks_cache_desc* caches, int32_t T,
+                                   const float* const* x0, const int32_t* const* w,
+                                   const double* const* t, const ks_params* params,
+                                   void* workspace, size_t workspace_bytes, ks_result* outs,
+                                   ks_stream_t stream);
+
+/*
  * Re-run check of one layer set (review: the DP keeps a single state per cell
  * with no optimality proof, referee major 1 on Eq. 8 / Algorithm 1 -- so a
  * chosen set is worth checking from scratch): the set's items run on x0 in

@@ -79,7 +79,8 @@ EXPORTS = ["ks_version", "ks_last_error", "ks_status_string", "ks_quantize_weigh
            "ks_select_step", "ks_reconstruct", "ks_tpt_argmax", "ks_solve", "ks_solve_cells",
            "ks_profile_start", "ks_profile_stop", "ks_reference_forward_noalloc",
            "ks_workspace_status", "ks_gemm_bf16", "ks_attention_bf16",
-           "ks_check_bounded_wait", "ks_lemma_workspace_size", "ks_lemma_check", "ks_eval_set"]
+           "ks_check_bounded_wait", "ks_lemma_workspace_size", "ks_lemma_check", "ks_eval_set",
+           "ks_workspace_size_contexts", "ks_solve_contexts"]
 
 _lib = None
 
@@ -118,6 +119,8 @@ def load() -> ctypes.CDLL:
         "ks_attention_bf16": ([P, P, P, I64, I32, I32, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "ks_profile_stop": ([P, I32, ctypes.POINTER(I32)], ctypes.c_int),
         "ks_eval_set": ([P, P, P, I32, P, P, P, P, P, P, SZ, P], ctypes.c_int),
+        "ks_workspace_size_contexts": ([P, I32, P, I32, ctypes.POINTER(SZ)], ctypes.c_int),
+        "ks_solve_contexts": ([P, P, I32, P, I32, P, P, P, P, P, SZ, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -519,6 +522,94 @@ class Solver:
         s = int(self.out.status.item())
         if s != 0:
             raise KnapSpecError(f"device status {s}: {load().ks_status_string(s).decode()}")
+
+
+class SolverContexts:
+    """The DP of one model at several contexts in one pass (ks_solve_contexts):
+    per context a KV cache view and context length, latencies (and optionally
+    weights); each context keeps its own result buffers (``outs[j]``, shaped as
+    a Solver's)."""
+
+    def __init__(self, model: ModelDesc, layers: Sequence[Dict[str, torch.Tensor]],
+                 caches: Sequence[tuple], T: int, ts: Sequence[Sequence[float]], prm: Params,
+                 ws: Optional[Sequence[Sequence[int]]] = None, keep_bp: bool = True,
+                 keep_cos: bool = False, keep_tpt: bool = True, keep_ref: bool = True,
+                 device="cuda", kv: str = "cache"):
+        """caches: per context (k_cache, v_cache, ctx)."""
+        n = len(caches)
+        if not 1 <= n <= 4:
+            raise KnapSpecError("1 to 4 contexts")
+        if len(ts) != n or (ws is not None and len(ws) != n):
+            raise KnapSpecError("one latency list (and weight list) per context")
+        self.model = model
+        self.wdtype = torch.float32 if model.wdtype == KS_F32 else torch.bfloat16
+        self._layers_keep = layers
+        self.layers = layer_array(layers, self.wdtype, model)
+        self._cache_keep = list(caches)
+        self.caches = (CacheDesc * n)(*[cache_desc(k, v, ctx, model, kv=kv) for k, v, ctx in caches])
+        self.n_ctx, self.T = n, T
+        self.n_items = 2 * model.n_layers
+        self.t = [list(map(float, t)) for t in ts]
+        for t in self.t:
+            if len(t) != self.n_items:
+                raise KnapSpecError("need one latency per item")
+        self.prm = prm
+        self.w = [list(ws[j]) if ws is not None else quantize_weights(self.t[j], prm.n_bins)
+                  for j in range(n)]
+        self.C = [solve_cells(self.t[j], prm, self.w[j]) for j in range(n)]
+        size = ctypes.c_size_t()
+        cells = (ctypes.c_int32 * n)(*self.C)
+        _check(load().ks_workspace_size_contexts(ctypes.byref(model), n, cells, T,
+                                                 ctypes.byref(size)))
+        self.ws = torch.empty(size.value, dtype=torch.uint8, device=device)
+        self.device = self.ws.device
+        words = (self.n_items + 63) // 64
+        z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=device)
+        self.outs = []
+        for C in self.C:
+            ni = self.n_items
+            self.outs.append(SolveOutputs(
+                status=z(1, dt=torch.int32), values=z(C, dt=torch.float32),
+                sets=z(C, words, dt=torch.int64), used_w=z(C, dt=torch.int32),
+                t_draft=z(C, dt=torch.float64), best=z(2, dt=torch.int32),
+                best_tpt=z(1, dt=torch.float64),
+                bp=z(ni, C, dt=torch.uint8) if keep_bp else None,
+                cos_skip=z(ni, C, dt=torch.float32) if keep_cos else None,
+                cos_exec=z(ni, C, dt=torch.float32) if keep_cos else None,
+                tpt=z(C, prm.gamma_max, dt=torch.float64) if keep_tpt else None,
+                ref_states=z(ni + 1, T, model.d_model, dt=torch.float32) if keep_ref else None,
+                exec_counts=z(ni, dt=torch.int32)))
+        p = lambda x: None if x is None else x.data_ptr()
+        self.results = (Result * n)(*[
+            Result(p(o.status), p(o.values), p(o.sets), p(o.used_w), p(o.t_draft), p(o.bp),
+                   p(o.cos_skip), p(o.cos_exec), p(o.tpt), p(o.best), p(o.best_tpt),
+                   p(o.ref_states), p(o.exec_counts), None, None) for o in self.outs])
+        self._t_arrs = [(ctypes.c_double * self.n_items)(*t) for t in self.t]
+        self._w_arrs = [(ctypes.c_int32 * self.n_items)(*w) for w in self.w]
+        self._t_ptrs = (ctypes.c_void_p * n)(*[ctypes.cast(a, ctypes.c_void_p) for a in self._t_arrs])
+        self._w_ptrs = (ctypes.c_void_p * n)(*[ctypes.cast(a, ctypes.c_void_p) for a in self._w_arrs])
+
+    def solve(self, x0s: Sequence[torch.Tensor]) -> List[SolveOutputs]:
+        """Enqueue the solve of every context on the current stream (x0s: one
+        [T][d] fp32 tensor per context)."""
+        if len(x0s) != self.n_ctx:
+            raise KnapSpecError("one x0 per context")
+        for x in x0s:
+            _shape(x, (self.T, self.model.d_model), "x0")
+        ptrs = (ctypes.c_void_p * self.n_ctx)(*[_dev(x, torch.float32, "x0") for x in x0s])
+        with torch.cuda.device(self.device):
+            _check(load().ks_solve_contexts(ctypes.byref(self.model), self.layers, self.n_ctx,
+                                            self.caches, self.T, ptrs, self._w_ptrs, self._t_ptrs,
+                                            ctypes.byref(self.prm), _dev(self.ws), self.ws.numel(),
+                                            self.results, _stream()))
+        return self.outs
+
+    def check_status(self) -> None:
+        for j, o in enumerate(self.outs):
+            s = int(o.status.item())
+            if s != 0:
+                raise KnapSpecError(f"context {j}: device status {s}: "
+                                    f"{load().ks_status_string(s).decode()}")
 
 
 def profile_start(timing: bool = True) -> None:

@@ -307,6 +307,98 @@ static ks_status reference_chain(const Ctx& c, const float* x0, float* ref) {
   return KS_OK;
 }
 
+// Item k on several contexts' batches at once (bf16 weights, tensor cores):
+// group g applies the item to E[g] states in[g] -> out[g] of context cs[g], with
+// the normalised operand already in that context's workspace (xh).  Every GEMM
+// runs once over all groups' rows, so the item's weights are read once for all
+// contexts; the attention runs once per context (each has its own context
+// length and cache).  A group's rows get exactly the arithmetic of a one-group
+// call: the same kernels, the same fixed-order sums.
+static ks_status sublayer_multi(const Ctx* const* cs, int n, int k, const float* const* in,
+                                const int* E, float* const* out) {
+  const Ctx& c0 = *cs[0];
+  const ks_model_desc* m = c0.m;
+  const int l = k / 2;
+  const ks_layer_weights& L = c0.layers[l];
+  const int d = m->d_model, qd = m->n_q_heads * m->head_dim, F = m->ffn;
+  const int kvd = m->n_kv_heads * m->head_dim;
+  const double ab = (double)act_bytes(c0.act);
+  double Rd = 0.0;
+  for (int g = 0; g < n; ++g) Rd += (double)E[g] * c0.T;
+  if (Rd <= 0.0) return KS_OK;
+  GemmGroupArg grp[kGemmMaxGroups];
+  auto groups = [&](auto&& fill) {
+    for (int g = 0; g < n; ++g) grp[g] = fill(g, *cs[g], E[g] * cs[g]->T);
+  };
+  if (k % 2 == 0) {
+    {
+      ProfScope ps(KK_GEMM_Q, c0.st, 2.0 * Rd * qd * d, (Rd * d + (double)qd * d) * ab + Rd * qd * ab);
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.xh, c.ws.q, nullptr, c.ws.rope, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.wq, nullptr, qd, d, EPI_ROPE_BF16, c0.T, m->head_dim,
+                            c0.status, c0.st));
+    }
+    const bool window = c0.cache->kv_mode == KS_KV_WINDOW;
+    if (window) {
+      ProfScope ps(KK_GEMM_KV, c0.st, 2.0 * 2.0 * Rd * kvd * d,
+                   (Rd * d + 2.0 * kvd * d) * ab + 2.0 * Rd * kvd * ab, 2);
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.xh, c.ws.kw, nullptr, c.ws.rope, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.wk, nullptr, kvd, d, EPI_ROPE_BF16, c0.T, m->head_dim,
+                            c0.status, c0.st));
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.xh, c.ws.vw, nullptr, nullptr, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.wv, nullptr, kvd, d, EPI_STORE_BF16, c0.T, m->head_dim,
+                            c0.status, c0.st));
+    }
+    for (int g = 0; g < n; ++g) {
+      const Ctx& c = *cs[g];
+      if (E[g] <= 0) continue;
+      const double T = c.T, ctx = c.cache->ctx, R = (double)E[g] * c.T;
+      const double keys = (double)E[g] * (T * ctx + T * (T + 1) / 2);
+      const double kv_bytes = window ? 2.0 * ctx * kvd * 2.0 + 2.0 * R * kvd * ab
+                                     : 2.0 * (ctx + T) * kvd * 2.0;
+      ProfScope ps(KK_ATTN, c.st, 4.0 * m->n_q_heads * m->head_dim * keys, 2.0 * R * qd * ab + kv_bytes);
+      const size_t layer_off = (size_t)l * c.cache->cache_rows * kvd * 2;
+      KS_TRY(tc_attention(c.ws.q, (const char*)c.cache->k_cache + layer_off,
+                          (const char*)c.cache->v_cache + layer_off, c.cache->cache_rows,
+                          E[g] * c.T, c.T, m->n_q_heads, m->n_kv_heads, m->head_dim, c.cache->ctx,
+                          c.ws.att, c.status, c.st, nullptr, window ? c.ws.kw : nullptr,
+                          window ? c.ws.vw : nullptr));
+    }
+    {
+      ProfScope ps(KK_GEMM_O, c0.st, 2.0 * Rd * d * qd, (Rd * qd + (double)d * qd) * ab + Rd * d * 8.0);
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.att, out[g], in[g], nullptr, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.wo, nullptr, d, qd, EPI_RESID_F32, c0.T, m->head_dim,
+                            c0.status, c0.st));
+    }
+  } else {
+    {
+      ProfScope ps(KK_GEMM_GATEUP, c0.st, 2.0 * Rd * 2.0 * F * d,
+                   (Rd * d + 2.0 * F * d) * ab + Rd * F * ab);
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.xh, c.ws.gb, nullptr, nullptr, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.w_gate, L.w_up, F, d, EPI_SWIGLU_BF16, c0.T, m->head_dim,
+                            c0.status, c0.st));
+    }
+    {
+      ProfScope ps(KK_GEMM_DOWN, c0.st, 2.0 * Rd * d * F, (Rd * F + (double)d * F) * ab + Rd * d * 8.0);
+      groups([&](int g, const Ctx& c, int R) {
+        return GemmGroupArg{c.ws.gb, out[g], in[g], nullptr, R};
+      });
+      KS_TRY(tc_gemm_groups(grp, n, L.w_down, nullptr, d, F, EPI_RESID_F32, c0.T, m->head_dim,
+                            c0.status, c0.st));
+    }
+  }
+  return KS_OK;
+}
+
 // ---------------------------------------------------------------- allocation-free variant
 // Scratch for ks_reference_forward_noalloc: a fixed device array that every GPU
 // loading this library holds until the process exits.  Host code must not use
@@ -523,14 +615,22 @@ ks_status ks_solve_cells(int32_t n_items, const int32_t* w, const double* t, con
   return KS_OK;
 }
 
-ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
-                   const ks_cache_desc* cache, int32_t T, const float* x0, const float* ref,
-                   const int32_t* w, const double* t, const ks_params* params, void* workspace,
-                   size_t workspace_bytes, ks_result* out, ks_stream_t stream) {
-  KS_TRY(check_model(model));
-  if (!t || !params || !out || !x0) return fail(KS_ERR_INVALID_ARG, "solve: NULL argument");
-  if (!out->status || !out->values || !out->sets || !out->best)
-    return fail(KS_ERR_INVALID_ARG, "solve: result needs status, values, sets and best");
+// ---------------------------------------------------------------- the DP over one or more contexts
+// One context of a solve: its cache (context length), evaluation tokens, item
+// weights and latencies, result buffers and its slice of the workspace.
+struct SolveCtx {
+  Ctx c;
+  const float* x0 = nullptr;
+  const float* ref = nullptr;
+  ks_result* out = nullptr;
+  std::vector<int32_t> w;
+  ItemTable tab;
+  int C = 0;
+  double t_target = 0.0;
+};
+
+static ks_status check_params(const ks_params* params) {
+  if (!params) return fail(KS_ERR_INVALID_ARG, "solve: params is NULL");
   if (params->gamma_max < 1 || !(params->alpha_scale > 0.0))
     return fail(KS_ERR_INVALID_ARG, "solve: gamma_max >= 1 and alpha_scale > 0");
   if (params->budget_mode != KS_BUDGET_AT_MOST && params->budget_mode != KS_BUDGET_EXACT)
@@ -539,129 +639,260 @@ ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
     return fail(KS_ERR_INVALID_ARG, "solve: prune_tau is NaN (use -INFINITY to turn it off)");
   if (params->dedup < 0 || params->dedup > 2)
     return fail(KS_ERR_INVALID_ARG, "solve: dedup must be 0 (off), 1 (on) or 2 (8-bit fingerprints)");
+  return KS_OK;
+}
+
+// Host checks of one context's inputs and results; its item weights (given, or
+// quantised from t) and grid size.
+static ks_status prepare_context(const ks_model_desc* model, const int32_t* w, const double* t,
+                                 const ks_params* params, const float* x0, const float* ref,
+                                 ks_result* out, SolveCtx* s) {
+  if (!t || !out || !x0) return fail(KS_ERR_INVALID_ARG, "solve: NULL argument");
+  if (!out->status || !out->values || !out->sets || !out->best)
+    return fail(KS_ERR_INVALID_ARG, "solve: result needs status, values, sets and best");
   KS_TRY(check_aligned16({x0, ref, out->ref_states, out->final_states}, "solve"));
   const int n_items = 2 * model->n_layers;
-  std::vector<int32_t> ww;
-  KS_TRY(resolve_weights(n_items, w, t, params, &ww));
-  ItemTable tab;
+  KS_TRY(resolve_weights(n_items, w, t, params, &s->w));
   long long K = 0;
   double t_target = 0.0;
   for (int i = 0; i < n_items; ++i) {
     if (!(t[i] > 0.0)) return fail(KS_ERR_INVALID_ARG, "solve: latencies must be positive");
-    tab.w[i] = ww[i];
-    tab.t[i] = t[i];
-    K += ww[i];
+    s->tab.w[i] = s->w[i];
+    s->tab.t[i] = t[i];
+    K += s->w[i];
     t_target += t[i];
   }
   if (K + 1 > (1 << 20)) return fail(KS_ERR_UNSUPPORTED, "more than 2^20 budget cells");
-  const int C = (int)(K + 1);
-  Ctx c;
-  KS_TRY(make_ctx(model, layers, cache, T, C + 1, workspace, workspace_bytes, (cudaStream_t)stream, &c));
-  c.status = out->status;
-  const cudaStream_t st = c.st;
-  const long long cell = (long long)T * model->d_model;
+  s->C = (int)(K + 1);
+  s->t_target = t_target;
+  s->x0 = x0;
+  s->ref = ref;
+  s->out = out;
+  return KS_OK;
+}
 
-  KS_CUDA_TRY(cudaMemsetAsync(out->status, 0, sizeof(int32_t), st));
-  if (cache->kv_mode == KS_KV_WINDOW && params->dedup) {
-    // rows past a compacted batch's live count are read (and masked) by the
-    // attention's window block: they must hold finite values from the start
-    const size_t kvb = (size_t)(C + 1) * T * model->n_kv_heads * model->head_dim *
-                       act_bytes(c.act);
-    KS_CUDA_TRY(cudaMemsetAsync(c.ws.kw, 0, kvb, st));
-    KS_CUDA_TRY(cudaMemsetAsync(c.ws.vw, 0, kvb, st));
-  }
-  {
-    ProfScope ps(KK_ROPE_TABLE, st, 0.0, 0.0);
-    KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, cache->ctx, model->rope_base, st));
-  }
+// The DP of n contexts that share the model's weights (one context: ks_solve).
+// Slot 0 of every state buffer carries the context's full-model state X^(k)
+// through the same batched kernels as its cells, so the select target X^(k+1)
+// comes out of each item's batch (exec slot 0) and no separate reference chain
+// runs.  Cells start from X^(0).  For every item, the contexts' batches go
+// through one grouped sublayer (tensor cores) and then one select each.
+static ks_status solve_run(const ks_model_desc* model, const ks_layer_weights* layers, int n,
+                           SolveCtx* ss, const ks_params* params) {
+  const int n_items = 2 * model->n_layers;
+  const cudaStream_t st = ss[0].c.st;
+  const int T = ss[0].c.T;
+  const long long cell = (long long)T * model->d_model;
   const double xb = model->wdtype == KS_F32 ? 4.0 : 2.0;
-  // Slot 0 of every state buffer carries the full model's state X^(k) through
-  // the same batched kernels as the cells, so the select target X^(k+1) comes
-  // out of each item's batch (exec slot 0) and no separate reference chain
-  // runs.  Cells start from X^(0).
   const bool dedup = params->dedup != 0;
-  if (dedup && C + 1 > 3072)
-    return fail(KS_ERR_UNSUPPORTED, "solve: distinct-state execution handles up to 3071 cells");
-  uint64_t* hprev = dedup ? c.ws.hash_a : nullptr;
-  uint64_t* hcur = dedup ? c.ws.hash_b : nullptr;
-  {
-    ProfScope ps(KK_BROADCAST, st, 0.0, (double)(C + 1) * cell * (4.0 + xb));
-    KS_TRY(launch_init_states(x0, C + 1, T, model->d_model, model->rms_eps, layers[0].attn_norm,
-                              model->wdtype, c.ws.prev, c.ws.xh, out->ref_states, hprev, st));
-  }
-  float* prev = c.ws.prev;
-  float* cur = c.ws.cur;
-  uint8_t* bp = out->bp ? out->bp : c.ws.bp;
   const bool exact = params->budget_mode == KS_BUDGET_EXACT;
   const bool pruning = params->prune_tau > -INFINITY || params->skip_cap >= 0;
   const bool track = exact || pruning;       // validity is carried only when it can change
-  uint8_t* vprev = track ? c.ws.valid_a : nullptr;
-  uint8_t* vcur = track ? c.ws.valid_b : nullptr;
-  if (track) KS_TRY(launch_init_valid(vprev, C, exact, st));
-  long long W_k = 0;                          // cumulative weight through item k
-  for (int k = 0; k < n_items; ++k) {
-    const int wk = ww[k];
-    const int E = C - wk;
-    W_k += wk;
-    const int min_valid_b =
-        params->skip_cap >= 0 ? (int)std::max(0LL, W_k - (long long)params->skip_cap) : 0;
-    if (dedup) {
-      // fold equal source states together, then run the item once per distinct state
-      {
-        ProfScope ps(KK_DEDUP, st, 0.0, (E + 1.0) * 9.0);
-        KS_TRY(launch_dedup(hprev, vprev, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
-                            out->exec_counts ? out->exec_counts + k : nullptr,
-                            params->dedup == 2, st));
-      }
-      {
-        ProfScope ps(KK_DEDUP_VERIFY, st, 0.0, 2.0 * (E + 1.0) * cell * 4.0);
-        KS_TRY(launch_dedup_verify(prev, cell, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
-                                   out->exec_counts ? out->exec_counts + k : nullptr,
-                                   out->dedup_rejected ? out->dedup_rejected + k : nullptr, st));
-      }
-      {
-        ProfScope ps(KK_GATHER, st, 0.0, 2.0 * (E + 1.0) * cell * (4.0 + xb));
-        KS_TRY(launch_gather(c.ws.uniq, c.ws.count, E + 1, cell, prev, c.ws.xh, c.act, c.ws.prev_c,
-                             c.ws.xh_c, st));
-      }
-      KS_TRY(sublayer(c, k, c.ws.prev_c, E + 1, c.ws.exec, /*xh_ready=*/true, c.ws.xh_c,
-                      c.ws.count));
-    } else {
-      if (out->exec_counts) KS_TRY(launch_fill_i32(out->exec_counts + k, E + 1, st));
-      KS_TRY(sublayer(c, k, prev, E + 1, c.ws.exec, /*xh_ready=*/true));
+  struct Run {
+    float* prev;
+    uint8_t *bp, *vprev, *vcur;
+    uint64_t *hprev, *hcur;
+    long long W_k;
+  };
+  std::vector<Run> run(n);
+  for (int j = 0; j < n; ++j) {
+    SolveCtx& s = ss[j];
+    Ctx& c = s.c;
+    ks_result* out = s.out;
+    c.status = out->status;
+    const int C = s.C;
+    if (dedup && C + 1 > 3072)
+      return fail(KS_ERR_UNSUPPORTED, "solve: distinct-state execution handles up to 3071 cells");
+    KS_CUDA_TRY(cudaMemsetAsync(out->status, 0, sizeof(int32_t), st));
+    if (c.cache->kv_mode == KS_KV_WINDOW && dedup) {
+      // rows past a compacted batch's live count are read (and masked) by the
+      // attention's window block: they must hold finite values from the start
+      const size_t kvb = (size_t)(C + 1) * T * model->n_kv_heads * model->head_dim *
+                         act_bytes(c.act);
+      KS_CUDA_TRY(cudaMemsetAsync(c.ws.kw, 0, kvb, st));
+      KS_CUDA_TRY(cudaMemsetAsync(c.ws.vw, 0, kvb, st));
     }
-    float* val = (k == n_items - 1) ? out->values : c.ws.val;
+    {
+      ProfScope ps(KK_ROPE_TABLE, st, 0.0, 0.0);
+      KS_TRY(launch_rope_table(c.ws.rope, T, model->head_dim, c.cache->ctx, model->rope_base, st));
+    }
+    Run& r = run[j];
+    r.hprev = dedup ? c.ws.hash_a : nullptr;
+    r.hcur = dedup ? c.ws.hash_b : nullptr;
+    {
+      ProfScope ps(KK_BROADCAST, st, 0.0, (double)(C + 1) * cell * (4.0 + xb));
+      KS_TRY(launch_init_states(s.x0, C + 1, T, model->d_model, model->rms_eps,
+                                layers[0].attn_norm, model->wdtype, c.ws.prev, c.ws.xh,
+                                out->ref_states, r.hprev, st));
+    }
+    // the cells' states are updated in place: a select writes slot b only when
+    // its execute candidate wins (every select block reads only its own slot)
+    r.prev = c.ws.prev;
+    r.bp = out->bp ? out->bp : c.ws.bp;
+    r.vprev = track ? c.ws.valid_a : nullptr;
+    r.vcur = track ? c.ws.valid_b : nullptr;
+    if (track) KS_TRY(launch_init_valid(r.vprev, C, exact, st));
+    r.W_k = 0;
+  }
+  const bool tc = use_tensor_cores(model);
+  std::vector<const Ctx*> cs(n);
+  std::vector<const float*> ins(n);
+  std::vector<float*> outs(n);
+  std::vector<int> Es(n);
+  for (int k = 0; k < n_items; ++k) {
+    // the item's batched forward over every context's executing cells
+    for (int j = 0; j < n; ++j) {
+      SolveCtx& s = ss[j];
+      Ctx& c = s.c;
+      Run& r = run[j];
+      const int E = s.C - s.w[k];
+      cs[j] = &c;
+      ins[j] = r.prev;
+      outs[j] = c.ws.exec;
+      Es[j] = E + 1;
+      if (dedup) {
+        // fold equal source states together, then run the item once per distinct state
+        ks_result* out = s.out;
+        {
+          ProfScope ps(KK_DEDUP, st, 0.0, (E + 1.0) * 9.0);
+          KS_TRY(launch_dedup(r.hprev, r.vprev, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
+                              out->exec_counts ? out->exec_counts + k : nullptr,
+                              params->dedup == 2, st));
+        }
+        {
+          ProfScope ps(KK_DEDUP_VERIFY, st, 0.0, 2.0 * (E + 1.0) * cell * 4.0);
+          KS_TRY(launch_dedup_verify(r.prev, cell, E + 1, c.ws.map, c.ws.uniq, c.ws.count,
+                                     out->exec_counts ? out->exec_counts + k : nullptr,
+                                     out->dedup_rejected ? out->dedup_rejected + k : nullptr, st));
+        }
+        {
+          ProfScope ps(KK_GATHER, st, 0.0, 2.0 * (E + 1.0) * cell * (4.0 + xb));
+          KS_TRY(launch_gather(c.ws.uniq, c.ws.count, E + 1, cell, r.prev, c.ws.xh, c.act,
+                               c.ws.prev_c, c.ws.xh_c, st));
+        }
+        KS_TRY(sublayer(c, k, c.ws.prev_c, E + 1, c.ws.exec, /*xh_ready=*/true, c.ws.xh_c,
+                        c.ws.count));
+      } else if (s.out->exec_counts) {
+        KS_TRY(launch_fill_i32(s.out->exec_counts + k, E + 1, st));
+      }
+    }
+    if (!dedup) {
+      if (tc) {
+        KS_TRY(sublayer_multi(cs.data(), n, k, ins.data(), Es.data(), outs.data()));
+      } else {
+        for (int j = 0; j < n; ++j)
+          KS_TRY(sublayer(*cs[j], k, ins[j], Es[j], outs[j], /*xh_ready=*/true));
+      }
+    }
+    // each context's select
     const void* g_next = nullptr;
     if (k + 1 < n_items) g_next = (k + 1) % 2 == 0 ? layers[(k + 1) / 2].attn_norm
                                                     : layers[(k + 1) / 2].mlp_norm;
-    const float* target = ref ? ref + (long long)(k + 1) * cell : nullptr;
-    ProfScope ps(KK_SELECT, st, 10.0 * (2.0 * C - wk) * cell,
-                 (3.0 * C - wk + 2.0) * cell * 4.0 + (g_next ? (C + 1.0) * cell * xb : 0.0));
-    KS_TRY(launch_select_fused(prev, c.ws.exec, target, C, T, model->d_model, wk, model->rms_eps,
-                               g_next, model->wdtype, cur, c.ws.xh, val, bp + (long long)k * C,
-                               out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
-                               out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
-                               out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr,
-                               vprev, vcur, params->prune_tau, min_valid_b,
-                               dedup ? c.ws.map : nullptr, hcur, st));
-    std::swap(prev, cur);
-    std::swap(vprev, vcur);
-    std::swap(hprev, hcur);
+    for (int j = 0; j < n; ++j) {
+      SolveCtx& s = ss[j];
+      Ctx& c = s.c;
+      Run& r = run[j];
+      ks_result* out = s.out;
+      const int C = s.C, wk = s.w[k];
+      r.W_k += wk;
+      const int min_valid_b =
+          params->skip_cap >= 0 ? (int)std::max(0LL, r.W_k - (long long)params->skip_cap) : 0;
+      float* val = (k == n_items - 1) ? out->values : c.ws.val;
+      const float* target = s.ref ? s.ref + (long long)(k + 1) * cell : nullptr;
+      ProfScope ps(KK_SELECT, st, 10.0 * (2.0 * C - wk) * cell,
+                   (3.0 * C - wk + 2.0) * cell * 4.0 + (g_next ? (C + 1.0) * cell * xb : 0.0));
+      KS_TRY(launch_select_fused(
+          r.prev, c.ws.exec, target, C, T, model->d_model, wk, model->rms_eps, g_next,
+          model->wdtype, r.prev, c.ws.xh, val, r.bp + (long long)k * C,
+          out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
+          out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
+          out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr, r.vprev,
+          r.vcur, params->prune_tau, min_valid_b, dedup ? c.ws.map : nullptr, r.hcur,
+          out->status, st));
+      std::swap(r.vprev, r.vcur);
+      std::swap(r.hprev, r.hcur);
+    }
   }
-  if (out->final_states)
-    KS_CUDA_TRY(cudaMemcpyAsync(out->final_states, prev + cell, (size_t)C * cell * sizeof(float),
-                                cudaMemcpyDeviceToDevice, st));
-  double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;
-  {
-    ProfScope ps(KK_RECONSTRUCT, st, 0.0, (double)n_items * C);
-    KS_TRY(launch_reconstruct(bp, nullptr, nullptr, &tab, n_items, C, out->sets, out->used_w, tdp,
-                              out->status, vprev, st));
+  for (int j = 0; j < n; ++j) {
+    SolveCtx& s = ss[j];
+    Ctx& c = s.c;
+    Run& r = run[j];
+    ks_result* out = s.out;
+    const int C = s.C;
+    if (out->final_states)
+      KS_CUDA_TRY(cudaMemcpyAsync(out->final_states, r.prev + cell,
+                                  (size_t)C * cell * sizeof(float), cudaMemcpyDeviceToDevice, st));
+    double* tdp = out->t_draft ? out->t_draft : c.ws.t_draft;
+    {
+      ProfScope ps(KK_RECONSTRUCT, st, 0.0, (double)n_items * C);
+      KS_TRY(launch_reconstruct(r.bp, nullptr, nullptr, &s.tab, n_items, C, out->sets,
+                                out->used_w, tdp, out->status, r.vprev, st));
+    }
+    ProfScope ps(KK_TPT, st, 0.0, (double)C * 12.0);
+    KS_TRY(launch_tpt(out->values, tdp, C, s.t_target, params->gamma_max, params->alpha_lo,
+                      params->alpha_scale, params->alpha_max, out->tpt, out->best, out->best_tpt,
+                      st));
   }
-  ProfScope ps(KK_TPT, st, 0.0, (double)C * 12.0);
-  KS_TRY(launch_tpt(out->values, tdp, C, t_target, params->gamma_max, params->alpha_lo,
-                    params->alpha_scale, params->alpha_max, out->tpt, out->best, out->best_tpt,
-                    st));
   return KS_OK;
+}
+
+ks_status ks_solve(const ks_model_desc* model, const ks_layer_weights* layers,
+                   const ks_cache_desc* cache, int32_t T, const float* x0, const float* ref,
+                   const int32_t* w, const double* t, const ks_params* params, void* workspace,
+                   size_t workspace_bytes, ks_result* out, ks_stream_t stream) {
+  KS_TRY(check_model(model));
+  KS_TRY(check_params(params));
+  SolveCtx s;
+  KS_TRY(prepare_context(model, w, t, params, x0, ref, out, &s));
+  KS_TRY(make_ctx(model, layers, cache, T, s.C + 1, workspace, workspace_bytes,
+                  (cudaStream_t)stream, &s.c));
+  return solve_run(model, layers, 1, &s, params);
+}
+
+ks_status ks_workspace_size_contexts(const ks_model_desc* model, int32_t n_ctx,
+                                     const int32_t* n_cells, int32_t T, size_t* bytes) {
+  KS_TRY(check_model(model));
+  KS_TRY(check_T(T));
+  if (!bytes || !n_cells) return fail(KS_ERR_INVALID_ARG, "workspace_size_contexts: NULL pointer");
+  if (n_ctx < 1 || n_ctx > kGemmMaxGroups)
+    return fail(KS_ERR_INVALID_ARG, "workspace_size_contexts: n_ctx must be in 1..4");
+  size_t total = 0;
+  for (int j = 0; j < n_ctx; ++j) {
+    if (n_cells[j] < 1) return fail(KS_ERR_INVALID_ARG, "n_cells must be >= 1");
+    total += align_up(carve(model, (long long)n_cells[j] + 1, T, nullptr).total);
+  }
+  *bytes = total;
+  return KS_OK;
+}
+
+ks_status ks_solve_contexts(const ks_model_desc* model, const ks_layer_weights* layers,
+                            int32_t n_ctx, const ks_cache_desc* caches, int32_t T,
+                            const float* const* x0, const int32_t* const* w,
+                            const double* const* t, const ks_params* params, void* workspace,
+                            size_t workspace_bytes, ks_result* outs, ks_stream_t stream) {
+  KS_TRY(check_model(model));
+  KS_TRY(check_params(params));
+  if (n_ctx < 1 || n_ctx > kGemmMaxGroups)
+    return fail(KS_ERR_INVALID_ARG, "solve_contexts: n_ctx must be in 1..4");
+  if (!caches || !x0 || !t || !outs) return fail(KS_ERR_INVALID_ARG, "solve_contexts: NULL argument");
+  if (params->dedup && n_ctx > 1)
+    return fail(KS_ERR_UNSUPPORTED, "solve_contexts: distinct-state execution runs one context at a time");
+  if (!workspace) return fail(KS_ERR_INVALID_ARG, "workspace is NULL");
+  std::vector<SolveCtx> ss(n_ctx);
+  size_t off = 0;
+  for (int j = 0; j < n_ctx; ++j) {
+    if (caches[j].kv_mode != caches[0].kv_mode)
+      return fail(KS_ERR_INVALID_ARG, "solve_contexts: every context needs the same kv_mode");
+    KS_TRY(prepare_context(model, w ? w[j] : nullptr, t[j], params, x0[j], nullptr, &outs[j],
+                           &ss[j]));
+    const size_t need = align_up(carve(model, (long long)ss[j].C + 1, T, nullptr).total);
+    if (off + need > workspace_bytes)
+      return fail(KS_ERR_WORKSPACE, "workspace too small for the contexts (see ks_workspace_size_contexts)");
+    KS_TRY(make_ctx(model, layers, &caches[j], T, ss[j].C + 1, (char*)workspace + off, need,
+                    (cudaStream_t)stream, &ss[j].c));
+    off += need;
+  }
+  return solve_run(model, layers, n_ctx, ss.data(), params);
 }
 
 ks_status ks_eval_set(const ks_model_desc* model, const ks_layer_weights* layers,

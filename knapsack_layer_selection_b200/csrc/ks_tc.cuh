@@ -37,6 +37,24 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
                   int32_t* status, cudaStream_t st, const int* dyn_cells = nullptr,
                   RowMaxArgs rowmax = RowMaxArgs{1.0f, nullptr});
 
+// Up to kGemmMaxGroups independent row groups multiplied by the same B (and
+// B2) in one launch: group g computes out_g = epi(A_g . B^T) for its M_g rows
+// (its own residual and RoPE table).  One tile walk covers every group's row
+// tiles, so a weight tile read once serves all groups; each output element is
+// the same fixed-order sum over K as in a one-group launch.
+constexpr int kGemmMaxGroups = 4;
+struct GemmGroupArg {
+  const void* A;
+  void* out;
+  const float* resid;
+  const float2* rope_cs;
+  int M;
+};
+ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B, const void* B2,
+                         int N, int K, int epi, int T, int head_dim, int32_t* status,
+                         cudaStream_t st, const int* dyn_cells = nullptr,
+                         RowMaxArgs rowmax = RowMaxArgs{1.0f, nullptr});
+
 // Tensor map of a row-major bf16 matrix [rows][cols] (row_stride elements apart)
 // read in boxes of box_rows x box_cols with the 128-byte swizzle; reads outside
 // [rows) x [cols) return zeros.

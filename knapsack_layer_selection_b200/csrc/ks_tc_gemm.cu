@@ -66,22 +66,32 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float (&v)
                       pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-struct GemmParams {
+// One row group of a launch: its rows are m-tiles tile_m0 .. tile_m0 + ceil(M/BM) - 1
+// of the walk.
+struct GemmGroupDev {
   void* out;
   const float* resid;
   const float2* rope_cs;
-  int32_t* status;
-  int M, N_out, K;
-  int tiles_m, tiles_n;
-  int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
-  int T, head_dim;
-  const int* dyn_cells; // optional device count: M = min(M, *dyn_cells * T) at run time
-  RowMaxArgs rowmax;    // EPI_ROWMAX only
+  int M;
+  int tile_m0;
 };
 
-// Tile t of the walk -> (m-tile, n-tile).  Tiles go in groups of group_m m-tiles;
-// inside a group the m index runs fastest, so the CTAs in flight share a few
-// weight tiles and the group's A rows stay in L2 while its weight columns stream.
+struct GemmParams {
+  int32_t* status;
+  int N_out, K;
+  int tiles_m, tiles_n;  // m-tiles of all row groups together
+  int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
+  int T, head_dim;
+  const int* dyn_cells; // optional device count (one row group only): M = min(M, *dyn_cells * T)
+  RowMaxArgs rowmax;    // EPI_ROWMAX only
+  int n_groups;
+  GemmGroupDev grp[kGemmMaxGroups];
+};
+
+// Tile t of the walk -> (m-tile of all row groups, n-tile).  Tiles go in groups
+// of group_m m-tiles; inside a group the m index runs fastest, so the CTAs in
+// flight share a few weight tiles and the group's A rows stay in L2 while its
+// weight columns stream.
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
   const int per_group = p.group_m * p.tiles_n;
   const int g = t / per_group;
@@ -92,16 +102,34 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm,
   tn = local / rows;
 }
 
+// m-tile of the walk -> (row group, m-tile inside it).
+__device__ __forceinline__ int tile_group(const GemmParams& p, int tm, int& local_tm) {
+  int g = 0, m0 = 0;
+#pragma unroll
+  for (int i = 1; i < kGemmMaxGroups; ++i)
+    if (i < p.n_groups && tm >= p.grp[i].tile_m0) {
+      g = i;
+      m0 = p.grp[i].tile_m0;
+    }
+  local_tm = tm - m0;
+  return g;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmA3,
+                   const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const GemmParams p_in) {
-  // rows can be decided on the device (a compacted batch): the walk uses the live count
+  // rows can be decided on the device (a compacted batch): the walk uses the live
+  // count.  Group fields are read from the parameter space (dynamically indexed);
+  // only group 0's row count can change, and it is kept in m_live0.
   GemmParams p = p_in;
+  int m_live0 = p_in.grp[0].M;
   if (p.dyn_cells) {
     const long long live = (long long)(*p.dyn_cells) * p.T;
-    p.M = (int)(live < p.M ? live : p.M);
-    p.tiles_m = (p.M + BM - 1) / BM;
+    m_live0 = (int)(live < m_live0 ? live : m_live0);
+    p.tiles_m = (m_live0 + BM - 1) / BM;
     if (p.group_m > p.tiles_m) p.group_m = p.tiles_m > 0 ? p.tiles_m : 1;
   }
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -127,6 +155,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
+    if (p.n_groups > 1) prefetch_tmap(&tmA1);
+    if (p.n_groups > 2) prefetch_tmap(&tmA2);
+    if (p.n_groups > 3) prefetch_tmap(&tmA3);
     prefetch_tmap(&tmB);
     if (EPI == EPI_SWIGLU_BF16) prefetch_tmap(&tmB2);
   }
@@ -145,8 +176,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        int tm, tn;
-        tile_coords(p, t, tm, tn);
+        int tmg, tn, tm;
+        tile_coords(p, t, tmg, tn);
+        const int grp = tile_group(p, tmg, tm);
+        const CUtensorMap* am = grp == 0 ? &tmA : grp == 1 ? &tmA1 : grp == 2 ? &tmA2 : &tmA3;
         const int m0 = tm * BM;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
@@ -159,7 +192,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a_dst = smem_u32(smem + s * STAGE_BYTES);
           const uint32_t b_dst = a_dst + A_BYTES;
           mbar_arrive_expect_tx(full, STAGE_BYTES);
-          tma_load_2d(a_dst, &tmA, kb * BK, m0, full);
+          tma_load_2d(a_dst, am, kb * BK, m0, full);
           if (EPI == EPI_SWIGLU_BF16) {
             tma_load_2d(b_dst, &tmB, kb * BK, tn * (BN / 2), full);
             tma_load_2d(b_dst + B_BYTES / 2, &tmB2, kb * BK, tn * (BN / 2), full);
@@ -217,11 +250,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got = mbar_wait(smem_u32(&tail->tfull[acc]), ar & 1u, abort, p.status);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      int tm, tn;
-      tile_coords(p, t, tm, tn);
+      int tmg, tn, tm;
+      tile_coords(p, t, tmg, tn);
+      const int gi = tile_group(p, tmg, tm);
+      const GemmGroupDev& gr = p_in.grp[gi];
+      void* const g_out = gr.out;
+      const float* const g_resid = gr.resid;
+      const float2* const g_rope = gr.rope_cs;
       const int m0 = tm * BM;
       const int row = m0 + q * 32 + lane;
-      const bool live = row < p.M;
+      const bool live = row < (gi == 0 ? m_live0 : gr.M);
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       float v[32], u[32];
       if (EPI == EPI_RESID_F32 || EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
@@ -233,11 +271,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!live) continue;
           const long long off = (long long)row * p.N_out + n0 + c * 32;
           if (EPI == EPI_STORE_BF16) {
-            store_bf16x32((__nv_bfloat16*)p.out + off, v);
+            store_bf16x32((__nv_bfloat16*)g_out + off, v);
           } else {
-            float4* o = reinterpret_cast<float4*>((float*)p.out + off);
+            float4* o = reinterpret_cast<float4*>((float*)g_out + off);
             if (EPI == EPI_RESID_F32) {
-              const float4* rr = reinterpret_cast<const float4*>(p.resid + off);
+              const float4* rr = reinterpret_cast<const float4*>(g_resid + off);
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const float4 x = rr[j];
@@ -274,7 +312,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         if (live)
-          reinterpret_cast<float4*>(p.out)[(long long)row * p.tiles_n + tn] =
+          reinterpret_cast<float4*>(g_out)[(long long)row * p.tiles_n + tn] =
               make_float4(v1, __int_as_float(i1), v2, 0.f);
       } else if (EPI == EPI_SWIGLU_BF16) {
         // columns 0..127: gate, 128..255: up, for output columns tn*128 ..
@@ -287,13 +325,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!live) continue;
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = v[j] / (1.0f + __expf(-v[j])) * u[j];
-          store_bf16x32((__nv_bfloat16*)p.out + (long long)row * p.N_out + n0 + c * 32, v);
+          store_bf16x32((__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + c * 32, v);
         }
       } else if (EPI == EPI_ROPE_BF16) {
         // rotate-half RoPE inside each head of this tile: column j pairs with j + hd/2
         const int half = p.head_dim / 2;
         const int tok = row % p.T;
-        const float2* cs = p.rope_cs + (long long)tok * half;
+        const float2* cs = g_rope + (long long)tok * half;
         const int n0 = tn * BN;
 #pragma unroll 1
         for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
@@ -310,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               v[j] = x1 * r.x - x2 * r.y;
               u[j] = x2 * r.x + x1 * r.y;
             }
-            __nv_bfloat16* o = (__nv_bfloat16*)p.out + (long long)row * p.N_out + n0 + h0 + c;
+            __nv_bfloat16* o = (__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + h0 + c;
             store_bf16x32(o, v);
             store_bf16x32(o + half, u);
           }
@@ -356,7 +394,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int EPI>
-ks_status launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+ks_status launch(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& b2,
                  const GemmParams& gp, cudaStream_t st) {
   static std::atomic<unsigned long long> attr_set{0};
   auto k = tc_gemm_kernel<EPI>;
@@ -366,7 +404,7 @@ ks_status launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
   }));
   const int n_tiles = gp.tiles_m * gp.tiles_n;
   const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
-  k<<<grid, THREADS, SMEM_BYTES, st>>>(a, b, b2, gp);
+  k<<<grid, THREADS, SMEM_BYTES, st>>>(a[0], a[1], a[2], a[3], b, b2, gp);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -396,17 +434,39 @@ bool use_tensor_cores(const ks_model_desc* m) { return m->wdtype == KS_BF16; }
 ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const float* resid,
                   int M, int N, int K, int epi, const float2* rope_cs, int T, int head_dim,
                   int32_t* status, cudaStream_t st, const int* dyn_cells, RowMaxArgs rowmax) {
-  if (M <= 0) return KS_OK;
+  const GemmGroupArg g{A, out, resid, rope_cs, M};
+  return tc_gemm_groups(&g, 1, B, B2, N, K, epi, T, head_dim, status, st, dyn_cells, rowmax);
+}
+
+ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B, const void* B2,
+                         int N, int K, int epi, int T, int head_dim, int32_t* status,
+                         cudaStream_t st, const int* dyn_cells, RowMaxArgs rowmax) {
+  if (n_groups < 1 || n_groups > kGemmMaxGroups)
+    return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: 1 to 4 row groups");
+  if (dyn_cells && n_groups != 1)
+    return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: a device row count needs one row group");
   if (K % BK) return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: K must be a multiple of 64");
   const int bn_out = epi == EPI_SWIGLU_BF16 ? BN / 2 : BN;
   if (N % bn_out)
     return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: N must be a multiple of " + std::to_string(bn_out));
-  if (epi == EPI_ROPE_BF16 && (head_dim % 64 || BN % head_dim || !rope_cs || T < 1))
-    return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: RoPE epilogue needs head_dim 64 or 128");
-  if (epi == EPI_RESID_F32 && !resid) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: resid is NULL");
   if (epi == EPI_SWIGLU_BF16 && !B2) return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: up weight is NULL");
-  CUtensorMap ta, tb, tb2;
-  KS_TRY(make_tmap_2d(&ta, A, M, K, K, BK, BM));
+  GemmParams gp{};
+  CUtensorMap ta[kGemmMaxGroups], tb, tb2;
+  int tiles_m = 0, n_live = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    const GemmGroupArg& a = groups[g];
+    if (a.M <= 0) continue;                     // an empty group takes no tiles
+    if (epi == EPI_ROPE_BF16 && (head_dim % 64 || BN % head_dim || !a.rope_cs || T < 1))
+      return fail(KS_ERR_UNSUPPORTED, "tensor-core GEMM: RoPE epilogue needs head_dim 64 or 128");
+    if (epi == EPI_RESID_F32 && !a.resid)
+      return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: resid is NULL");
+    KS_TRY(make_tmap_2d(&ta[n_live], a.A, a.M, K, K, BK, BM));
+    gp.grp[n_live] = GemmGroupDev{a.out, a.resid, a.rope_cs, a.M, tiles_m};
+    tiles_m += (a.M + BM - 1) / BM;
+    ++n_live;
+  }
+  if (n_live == 0) return KS_OK;
+  for (int g = n_live; g < kGemmMaxGroups; ++g) ta[g] = ta[0];
   if (epi == EPI_SWIGLU_BF16) {
     KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN / 2));
     KS_TRY(make_tmap_2d(&tb2, B2, N, K, K, BK, BN / 2));
@@ -414,15 +474,11 @@ ks_status tc_gemm(const void* A, const void* B, const void* B2, void* out, const
     KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN));
     tb2 = tb;
   }
-  GemmParams gp;
-  gp.out = out;
-  gp.resid = resid;
-  gp.rope_cs = rope_cs;
+  gp.n_groups = n_live;
   gp.status = status;
-  gp.M = M;
   gp.N_out = N;
   gp.K = K;
-  gp.tiles_m = (M + BM - 1) / BM;
+  gp.tiles_m = tiles_m;
   gp.tiles_n = N / bn_out;
   // a group's A rows (group_m x 128 rows x K) should stay well inside one die's
   // half of L2 (~32 MB) while the weight columns stream past them

@@ -304,3 +304,36 @@ def test_window_reading_and_dedup_mode_are_checked_before_any_launch(lib):
                       ctypes.byref(res), None)
     assert st == 1 and b"dedup must be" in lib.ks_last_error()
     assert B.params(4, 8, dedup="weak").dedup == 2 and B.params(4, 8, dedup=True).dedup == 1
+
+
+def test_solve_contexts_checks_before_any_launch(lib):
+    """ks_solve_contexts: 1..4 contexts, one key/value reading for all, no
+    distinct-state execution across contexts, a workspace sized by
+    ks_workspace_size_contexts -- all refused on the host."""
+    m = B.model_desc(1, 64, 1, 1, 64, 64, 1e-6, 1e4, "f32")
+    layers = (B.LayerWeights * 1)()
+    for f, _ in B.LayerWeights._fields_:
+        setattr(layers[0], f, 256)
+    p = ctypes.c_void_p(256)
+    t = (ctypes.c_double * 2)(1.0, 1.0)
+    tp = (ctypes.c_void_p * 2)(ctypes.cast(t, ctypes.c_void_p), ctypes.cast(t, ctypes.c_void_p))
+    x0 = (ctypes.c_void_p * 2)(256, 256)
+    caches = (B.CacheDesc * 2)(B.CacheDesc(256, 256, 16, 8), B.CacheDesc(256, 256, 16, 4))
+    res = (B.Result * 2)(B.Result(*([256] * 15)), B.Result(*([256] * 15)))
+    prm = B.params(4, 8)
+    call = lambda n, prm_, ws_bytes, cs=caches: lib.ks_solve_contexts(
+        ctypes.byref(m), layers, n, cs, 4, x0, None, tp, ctypes.byref(prm_), p, ws_bytes, res, None)
+    assert call(0, prm, 1 << 40) == 1 and b"n_ctx" in lib.ks_last_error()
+    assert call(5, prm, 1 << 40) == 1 and b"n_ctx" in lib.ks_last_error()
+    dd = B.params(4, 8, dedup=True)
+    assert call(2, dd, 1 << 40) == 2 and b"one context at a time" in lib.ks_last_error()
+    mixed = (B.CacheDesc * 2)(B.CacheDesc(256, 256, 16, 8, 0), B.CacheDesc(256, 256, 16, 8, 1))
+    assert call(2, prm, 1 << 40, mixed) == 1 and b"same kv_mode" in lib.ks_last_error()
+    assert call(2, prm, 1024) == 3 and b"workspace" in lib.ks_last_error()
+    # the workspace of several contexts is the sum of the one-context sizes
+    cells = (ctypes.c_int32 * 2)(9, 33)
+    size = ctypes.c_size_t()
+    assert lib.ks_workspace_size_contexts(ctypes.byref(m), 2, cells, 4, ctypes.byref(size)) == 0
+    one = [B.workspace_size(m, c, 4) for c in (9, 33)]
+    assert sum(one) <= size.value <= sum(one) + 512
+    assert lib.ks_workspace_size_contexts(ctypes.byref(m), 5, cells, 4, ctypes.byref(size)) == 1
