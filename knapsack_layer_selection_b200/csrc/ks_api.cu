@@ -807,8 +807,7 @@ static ks_status solve_run(const ks_model_desc* model, const ks_layer_weights* l
           out->cos_skip ? out->cos_skip + (long long)k * C : nullptr,
           out->cos_exec ? out->cos_exec + (long long)k * C : nullptr,
           out->ref_states ? out->ref_states + (long long)(k + 1) * cell : nullptr, r.vprev,
-          r.vcur, params->prune_tau, min_valid_b, dedup ? c.ws.map : nullptr, r.hcur,
-          out->status, st));
+          r.vcur, params->prune_tau, min_valid_b, dedup ? c.ws.map : nullptr, r.hcur, st));
       std::swap(r.vprev, r.vcur);
       std::swap(r.hprev, r.hcur);
     }

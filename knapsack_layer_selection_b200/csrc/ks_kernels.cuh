@@ -56,14 +56,12 @@ ks_status launch_select(const float* prev, const float* exec, const float* targe
 // valid_prev / valid_cur (both NULL: every cell valid) carry the exact-budget
 // validity of the cells from row to row.  cur may equal prev (the states are
 // then updated in place: a cell whose skip candidate wins is not rewritten).
-// A bounded wait that gives up reports KS_ERR_TIMEOUT in *status.
 ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
                               uint8_t* valid_cur, double prune_tau, int min_valid_b,
-                              const int* exec_map, uint64_t* hash_cur, int32_t* status,
-                              cudaStream_t st);
+                              const int* exec_map, uint64_t* hash_cur, cudaStream_t st);
 
 // Slots 0..n_slots-1 of a state buffer <- x0, and their normalised operands.
 ks_status launch_init_states(const float* x0, int n_slots, int T, int d, float eps, const void* g,

@@ -3,10 +3,8 @@
 // search (Eq. 4, Eq. 5) -- KnapSpec review page, referee major 1 and minor 4,
 // "What carries the argument".
 #include "ks_kernels.cuh"
-#include "ks_sm100.cuh"
 
 #include <float.h>
-#include <atomic>
 #include <type_traits>
 #include <math.h>
 
@@ -327,333 +325,14 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_fused_kernel(
   if (hash_cur) block_hash_store(hh, hash_sh, hash_cur + slot);
 }
 
-// ---------------------------------------------------------------- fused select, one cluster per cell
-// The same select as select_fused_kernel, with the cell's data staged on chip:
-// a cluster of kSelCL CTAs takes one slot (slot 0 = reference, slot b+1 = cell
-// b), and CTA `rank` takes tokens [rank*tpc, rank*tpc + tpc).  Each CTA copies
-// its tokens' rows of the skip candidate, the execute candidate and the target
-// into shared memory with bulk copies (one bounded mbarrier wait), sums the
-// per-token dot products from there, and sends its tokens' cosines to every
-// CTA of the cluster (distributed shared memory).  After a cluster barrier all
-// CTAs hold the T cosines, take the same decision (the mean is summed in token
-// order, as in select_fused_kernel), and each stores its tokens' winning rows
-// from shared memory: the state by bulk copy, the next item's normalised
-// operand from registers.  Every candidate byte is read from HBM once.
-// Barriers: the cluster barrier is reached by every thread of every CTA on
-// every path (a CTA whose copies timed out carries on with an error status),
-// and no CTA touches another's shared memory after the second barrier, so a
-// CTA may leave as soon as its own bulk stores have completed.
-constexpr int kSelCL = 8;
-constexpr int kSelClThreads = 256;
-
-struct SelClTail {
-  uint64_t full;
-  int abort;
-  int take;
-  uint32_t hash[2];
-  double cs[kSelectMaxT];
-  double ce[kSelectMaxT];
-  float inv_s[kSelectMaxT];
-  float inv_e[kSelectMaxT];
-  double red[kSelClThreads / 32][5];
-};
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// fp64 store into the shared memory of CTA `rank` of this cluster, at the
-// address that `local` has in this CTA
-__device__ __forceinline__ void st_cluster_f64(const void* local, uint32_t rank, double v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(remote)
-               : "r"(sm100::smem_u32(local)), "r"(rank));
-  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(remote), "d"(v) : "memory");
-}
-// bulk copy global -> this CTA's shared memory, completion counted on `bar`
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          sm100::smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-// bulk copy shared -> global (bulk-group completion)
-__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(sm100::smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_and_wait_all() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-template <typename TX, typename TG>
-__global__ void __cluster_dims__(kSelCL, 1, 1) __launch_bounds__(kSelClThreads)
-    select_cluster_kernel(const float* __restrict__ prev, const float* __restrict__ exec,
-                          const float* __restrict__ target_in, int T, int d, int w, float eps,
-                          const TG* __restrict__ g_next, float* __restrict__ cur,
-                          TX* __restrict__ xh_next, float* __restrict__ val,
-                          uint8_t* __restrict__ bp, float* __restrict__ cos_s_out,
-                          float* __restrict__ cos_e_out, float* __restrict__ ref_out,
-                          const uint8_t* __restrict__ valid_prev, uint8_t* __restrict__ valid_cur,
-                          double prune_tau, int min_valid_b, const int* __restrict__ exec_map,
-                          uint64_t* __restrict__ hash_cur, int32_t* __restrict__ status, int tpc) {
-  using namespace sm100;
-  extern __shared__ __align__(128) unsigned char smem[];
-  const long long cell = (long long)T * d;
-  const uint32_t rank = cluster_rank();
-  const int slot_i = (int)(blockIdx.x / kSelCL);
-  const bool is_ref = slot_i == 0;
-  const int b = slot_i - 1;
-  const int t0 = (int)rank * tpc;
-  const int nt = max(0, min(T, t0 + tpc) - t0);
-  float* s_buf = reinterpret_cast<float*>(smem);          // [tpc][d] skip (or kept) rows
-  float* e_buf = s_buf + (long long)tpc * d;             // [tpc][d] execute rows
-  float* r_buf = e_buf + (long long)tpc * d;             // [tpc][d] target rows
-  SelClTail* tl = reinterpret_cast<SelClTail*>(r_buf + (long long)tpc * d);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  int e_idx = b - w + 1;
-  if (exec_map && !is_ref && b >= w) e_idx = exec_map[b - w + 1];
-  const bool has_e = !is_ref && b >= w && e_idx >= 0;
-  const float* s_base = is_ref ? exec : prev + (long long)(b + 1) * cell;
-  const float* e_base = has_e ? exec + (long long)e_idx * cell : nullptr;
-  const float* target = target_in ? target_in : exec;
-  const long long slot = is_ref ? 0 : (long long)(b + 1);
-
-  if (tid == 0) {
-    mbar_init(smem_u32(&tl->full), 1);
-    tl->abort = 0;
-    tl->hash[0] = tl->hash[1] = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  cluster_arrive_relaxed();                      // peers may write our cosines after the wait below
-
-  const uint32_t row_bytes = (uint32_t)d * 4u;
-  const uint32_t full = smem_u32(&tl->full);
-  if (tid == 0 && nt > 0) {
-    const uint32_t per = 1u + (is_ref ? 0u : 1u) + (has_e ? 1u : 0u);
-    mbar_arrive_expect_tx(full, per * (uint32_t)nt * row_bytes);
-    for (int i = 0; i < nt; ++i) {
-      const long long off = (long long)(t0 + i) * d;
-      bulk_load(s_buf + (long long)i * d, s_base + off, row_bytes, full);
-      if (!is_ref) bulk_load(r_buf + (long long)i * d, target + off, row_bytes, full);
-      if (has_e) bulk_load(e_buf + (long long)i * d, e_base + off, row_bytes, full);
-    }
-  }
-  bool ok = true;
-  if (nt > 0) ok = mbar_wait(full, 0, &tl->abort, status);
-
-  // per-token sums: thread i takes float4 columns i, i + 256, ... (fp32 partials of four
-  // products accumulated in fp64), then warps in shuffle order, then warps in index order
-  const int d4 = d / 4;
-  for (int i = 0; i < nt; ++i) {
-    const float4* s4 = reinterpret_cast<const float4*>(s_buf + (long long)i * d);
-    const float4* r4 = reinterpret_cast<const float4*>(r_buf + (long long)i * d);
-    const float4* e4 = reinterpret_cast<const float4*>(e_buf + (long long)i * d);
-    double sr = 0, ss = 0, rr = 0, er = 0, ee = 0;
-    if (ok) {
-      for (int j = tid; j < d4; j += kSelClThreads) {
-        const float4 a = s4[j];
-        ss += (double)dot4(a, a);
-        if (!is_ref) {
-          const float4 r = r4[j];
-          sr += (double)dot4(a, r);
-          rr += (double)dot4(r, r);
-          if (has_e) {
-            const float4 e = e4[j];
-            er += (double)dot4(e, r);
-            ee += (double)dot4(e, e);
-          }
-        }
-      }
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      sr += __shfl_xor_sync(0xffffffffu, sr, o);
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      rr += __shfl_xor_sync(0xffffffffu, rr, o);
-      er += __shfl_xor_sync(0xffffffffu, er, o);
-      ee += __shfl_xor_sync(0xffffffffu, ee, o);
-    }
-    if (lane == 0) {
-      tl->red[warp][0] = sr;
-      tl->red[warp][1] = ss;
-      tl->red[warp][2] = rr;
-      tl->red[warp][3] = er;
-      tl->red[warp][4] = ee;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      double a[5] = {0, 0, 0, 0, 0};
-      for (int q = 0; q < kSelClThreads / 32; ++q)
-        for (int c = 0; c < 5; ++c) a[c] += tl->red[q][c];
-      const int t = t0 + i;
-      tl->cs[t] = is_ref ? 0.0 : a[0] / sqrt(a[1] * a[2]);
-      tl->ce[t] = has_e ? a[3] / sqrt(a[4] * a[2]) : 0.0;
-      tl->inv_s[t] = (float)(1.0 / sqrt(a[1] / (double)d + (double)eps));
-      tl->inv_e[t] = (float)(1.0 / sqrt(a[4] / (double)d + (double)eps));
-    }
-    __syncthreads();
-  }
-
-  cluster_wait();                                // every CTA of the cluster is running
-  if (tid < kSelCL && !is_ref) {
-    // thread q sends this CTA's token cosines to CTA q (itself included)
-    for (int i = 0; i < nt; ++i) {
-      const int t = t0 + i;
-      st_cluster_f64(&tl->cs[t], (uint32_t)tid, tl->cs[t]);
-      st_cluster_f64(&tl->ce[t], (uint32_t)tid, tl->ce[t]);
-    }
-  }
-  cluster_arrive();
-  cluster_wait();                                // all T cosines are here; no remote access after
-
-  if (tid == 0) {
-    int take = 0;
-    if (!is_ref) {
-      double ms = 0.0, me = 0.0;
-      for (int t = 0; t < T; ++t) {
-        ms += tl->cs[t];
-        me += tl->ce[t];
-      }
-      ms /= (double)T;
-      me /= (double)T;
-      const bool sv = valid_prev ? valid_prev[b] != 0 : true;
-      const bool ev = has_e && (valid_prev ? valid_prev[b - w] != 0 : true);
-      take = ev && (!sv || me > ms) ? 1 : 0;
-      const double kept = take ? me : ms;
-      const bool alive = (sv || ev) && !(kept < prune_tau) && b >= min_valid_b;
-      if (rank == 0) {
-        const float nan = __int_as_float(0x7fc00000);
-        val[b] = alive ? (float)kept : nan;
-        bp[b] = (uint8_t)take;
-        if (valid_cur) valid_cur[b] = (uint8_t)alive;
-        if (cos_s_out) cos_s_out[b] = sv ? (float)ms : nan;
-        if (cos_e_out) cos_e_out[b] = ev ? (float)me : nan;
-      }
-    }
-    tl->take = take;
-  }
-  __syncthreads();
-  const bool take = tl->take != 0;
-  const float* src = take ? e_buf : s_buf;
-  const float* inv = take ? tl->inv_e : tl->inv_s;
-  if (tid == 0 && nt > 0 && ok) {
-    // the state rows, straight from shared memory (in place, a kept skip state stays put)
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const uint32_t bytes = (uint32_t)nt * row_bytes;
-    if (!(cur == prev && !is_ref && !take))
-      bulk_store(cur + slot * cell + (long long)t0 * d, src, bytes);
-    if (is_ref && ref_out) bulk_store(ref_out + (long long)t0 * d, src, bytes);
-  }
-  Hash2 hh;
-  if (ok && (g_next || hash_cur)) {
-    TX* xdst = g_next ? xh_next + slot * cell + (long long)t0 * d : nullptr;
-    const float4* src4 = reinterpret_cast<const float4*>(src);
-    const int n4 = nt * d4;
-    for (int i = tid; i < n4; i += kSelClThreads) {
-      const float4 v = src4[i];
-      const int tl_i = i / d4;
-      const int j = (i - tl_i * d4) * 4;
-      if (hash_cur) hh.add4(v, (uint32_t)((long long)(t0 + tl_i) * d + j));
-      if (xdst) store_norm4(xdst + (long long)i * 4, v, inv[t0 + tl_i], g_next + j);
-    }
-  }
-  if (hash_cur) {
-    // this CTA's share of the order-independent fingerprint, added into the slot's word
-    for (int o = 16; o > 0; o >>= 1) {
-      hh.a += __shfl_xor_sync(0xffffffffu, hh.a, o);
-      hh.b += __shfl_xor_sync(0xffffffffu, hh.b, o);
-    }
-    if (lane == 0) {
-      atomicAdd(&tl->hash[0], hh.a);
-      atomicAdd(&tl->hash[1], hh.b);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t* hw = reinterpret_cast<uint32_t*>(hash_cur + slot);   // little-endian: [1] = high
-      atomicAdd(hw + 1, tl->hash[0]);
-      atomicAdd(hw, tl->hash[1]);
-    }
-  }
-  if (tid == 0) {
-    bulk_commit_and_wait_all();                  // the state stores have left shared memory
-    if (!ok && nt > 0) mbar_wait_drain(full, 0, status);   // never leave under a landing copy
-  }
-}
-
-// Zeroes the fingerprint words the cluster select adds into (one per slot).
-__global__ void zero_u64_kernel(uint64_t* p, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) p[i] = 0;
-}
-
-// Shared memory of one cluster-select CTA for T tokens of width d, or 0 when
-// its rows do not fit two CTAs to an SM.
-static size_t select_cluster_smem(int T, int d) {
-  const int tpc = (T + kSelCL - 1) / kSelCL;
-  const size_t bytes = 3ull * tpc * d * 4 + sizeof(SelClTail);
-  return bytes <= 110u * 1024u ? bytes : 0;
-}
-
 ks_status launch_select_fused(const float* prev, const float* exec, const float* target, int C,
                               int T, int d, int w, float eps, const void* g_next, int wdt,
                               float* cur, void* xh_next, float* val, uint8_t* bp, float* cos_s,
                               float* cos_e, float* ref_out, const uint8_t* valid_prev,
                               uint8_t* valid_cur, double prune_tau, int min_valid_b,
-                              const int* exec_map, uint64_t* hash_cur, int32_t* status,
-                              cudaStream_t st) {
+                              const int* exec_map, uint64_t* hash_cur, cudaStream_t st) {
   if (T > kSelectMaxT) return fail(KS_ERR_UNSUPPORTED, "select: T above 256");
   if (d % 4 != 0) return fail(KS_ERR_UNSUPPORTED, "select: d must be a multiple of 4");
-  const size_t csm = select_cluster_smem(T, d);
-  if (csm) {
-    const int tpc = (T + kSelCL - 1) / kSelCL;
-    static std::atomic<unsigned long long> attr_bf{0}, attr_f{0};
-    if (hash_cur) {
-      zero_u64_kernel<<<ceil_div(C + 1, 256), 256, 0, st>>>(hash_cur, C + 1);
-      KS_LAUNCH_CHECK();
-    }
-    const dim3 grid((unsigned)(C + 1) * kSelCL);
-    if (wdt == KS_BF16) {
-      auto k = select_cluster_kernel<__nv_bfloat16, __nv_bfloat16>;
-      KS_TRY(once_per_device(attr_bf, [&]() -> ks_status {
-        KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024));
-        return KS_OK;
-      }));
-      k<<<grid, kSelClThreads, csm, st>>>(prev, exec, target, T, d, w, eps,
-                                          (const __nv_bfloat16*)g_next, cur,
-                                          (__nv_bfloat16*)xh_next, val, bp, cos_s, cos_e, ref_out,
-                                          valid_prev, valid_cur, prune_tau, min_valid_b, exec_map,
-                                          hash_cur, status, tpc);
-    } else {
-      auto k = select_cluster_kernel<float, float>;
-      KS_TRY(once_per_device(attr_f, [&]() -> ks_status {
-        KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024));
-        return KS_OK;
-      }));
-      k<<<grid, kSelClThreads, csm, st>>>(prev, exec, target, T, d, w, eps, (const float*)g_next,
-                                          cur, (float*)xh_next, val, bp, cos_s, cos_e, ref_out,
-                                          valid_prev, valid_cur, prune_tau, min_valid_b, exec_map,
-                                          hash_cur, status, tpc);
-    }
-    KS_LAUNCH_CHECK();
-    return KS_OK;
-  }
   if (wdt == KS_BF16)
     select_fused_kernel<__nv_bfloat16, __nv_bfloat16><<<C + 1, kSelectThreads, 0, st>>>(
         prev, exec, target, T, d, w, eps, (const __nv_bfloat16*)g_next, cur,

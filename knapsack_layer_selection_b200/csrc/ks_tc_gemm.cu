@@ -81,6 +81,7 @@ struct GemmParams {
   int N_out, K;
   int tiles_m, tiles_n;  // m-tiles of all row groups together
   int group_m;          // tile walk: groups of group_m m-tiles, m fastest inside a group
+  int group_n;          // > 0: bands of group_n n-tiles instead, n fastest inside a band
   int T, head_dim;
   const int* dyn_cells; // optional device count (one row group only): M = min(M, *dyn_cells * T)
   RowMaxArgs rowmax;    // EPI_ROWMAX only
@@ -93,6 +94,18 @@ struct GemmParams {
 // flight share a few weight tiles and the group's A rows stay in L2 while its
 // weight columns stream.
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm, int& tn) {
+  if (p.group_n > 0) {
+    // a band of group_n weight tiles stays in L2 while every row tile passes it
+    // once; the CTAs in flight read the same activation tile at about the same time
+    const int per_band = p.group_n * p.tiles_m;
+    const int g = t / per_band;
+    const int local = t - g * per_band;
+    const int n_base = g * p.group_n;
+    const int cols = min(p.group_n, p.tiles_n - n_base);
+    tn = n_base + local % cols;
+    tm = local / cols;
+    return;
+  }
   const int per_group = p.group_m * p.tiles_n;
   const int g = t / per_group;
   const int local = t - g * per_group;
@@ -480,14 +493,29 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
   gp.K = K;
   gp.tiles_m = tiles_m;
   gp.tiles_n = N / bn_out;
-  // a group's A rows (group_m x 128 rows x K) should stay well inside one die's
-  // half of L2 (~32 MB) while the weight columns stream past them
+  // Tile walk: either groups of group_m row tiles whose A rows (group_m x 128 x K,
+  // at most ~32 MB, well inside one die's half of L2) stay resident while the
+  // weight columns stream past them -- B is then read once per group -- or bands
+  // of group_n weight tiles (at most ~48 MB of B) that stay resident while every
+  // row tile passes -- A is then read once per band.  The walk with the smaller
+  // estimated DRAM traffic is taken (a long-K, narrow-N product like the MLP's
+  // down projection reads its weights ~8 times under the first and A twice under
+  // the second).  The walk changes only which CTA computes a tile and when, never
+  // a tile's arithmetic.
   {
     const long long a_tile = (long long)BM * K * 2;
+    const long long b_tile = (long long)BN * K * 2;
     long long g = (32ll << 20) / a_tile;
     if (g < 8) g = 8;
     if (g > 32) g = 32;
     gp.group_m = (int)(g < gp.tiles_m ? g : gp.tiles_m);
+    long long h = (48ll << 20) / b_tile;
+    if (h < 1) h = 1;
+    if (h > gp.tiles_n) h = gp.tiles_n;
+    const long long a_all = a_tile * gp.tiles_m, b_all = b_tile * gp.tiles_n;
+    const long long by_m = a_all + b_all * ((gp.tiles_m + gp.group_m - 1) / gp.group_m);
+    const long long by_n = b_all + a_all * ((gp.tiles_n + h - 1) / h);
+    gp.group_n = (epi != EPI_ROWMAX && !dyn_cells && by_n < by_m) ? (int)h : 0;
   }
   gp.T = T;
   gp.head_dim = head_dim;

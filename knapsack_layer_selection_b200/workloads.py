@@ -211,6 +211,16 @@ def window_weights(wl: Workload, seed: int = 2, device: Optional[str] = None
             for _ in range(wl.n_layers)]
 
 
+def sequence_embeddings(wl: Workload, seed: int = 3, device: Optional[str] = None) -> torch.Tensor:
+    """N(0, 1) input embeddings [ctx + T][d] fp32 of a whole token sequence, from
+    their own generator and seed: the input of a full-model prefill, whose last T
+    rows are then the evaluation tokens' x0."""
+    dev = device or wl.gen_device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    return _randn((wl.n_positions, wl.d_model), 1.0, torch.float32, gen, dev)
+
+
 def truncated(wl: Workload, n_layers: int, ctx: Optional[int] = None) -> Workload:
     """The same workload shape with fewer layers (and optionally another context)."""
     return dataclasses.replace(wl, n_layers=n_layers, ctx=wl.ctx if ctx is None else ctx)

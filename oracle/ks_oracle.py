@@ -624,6 +624,63 @@ def scalar_knapsack_dp(w: Sequence[int], v: Sequence[int], capacity: int,
 
 
 # --------------------------------------------------------------------------
+# The full model's prefill: the KV cache "from the full model"
+# --------------------------------------------------------------------------
+@dataclass
+class Prefill:
+    k_cache: np.ndarray    # [L, n, Hkv, hd] rotated keys of every position
+    v_cache: np.ndarray    # [L, n, Hkv, hd]
+    hidden: np.ndarray     # [2L+1, n, d] residual stream after each item (row 0 = emb)
+
+
+def prefill(model: Model, emb: np.ndarray) -> Prefill:
+    """Run the full decoder over a token sequence emb [n, d] (positions 0 .. n-1)
+    with causal self-attention, recording each layer's keys and values.
+
+    This is how the workloads' "KV cache from the full model" is produced for the
+    small configurations: the cache the DP reads (reading R7) holds what the
+    unpruned model computed for every position, the evaluation tokens' included.
+    Per layer (the same sublayer definitions as attn_item / mlp_item): x^ =
+    RMSNorm(h); q = RoPE(x^ Wq^T), k = RoPE(x^ Wk^T) and v = x^ Wv^T at each
+    token's own position (reading R8); position i attends to positions 0 .. i,
+    query head h to kv head h // (Hq / Hkv); h += o Wo^T; then the MLP item.
+    Needs Wk / Wv in every layer.
+    """
+    h = np.asarray(emb, F64)
+    n, d = h.shape
+    L = len(model.layers)
+    Hq, Hkv, hd = model.n_q_heads, model.n_kv_heads, model.head_dim
+    group = Hq // Hkv
+    pos = np.arange(n)
+    causal = pos[None, :] <= pos[:, None]                      # [query, key]
+    kc = np.empty((L, n, Hkv, hd))
+    vc = np.empty((L, n, Hkv, hd))
+    hidden = [h]
+    for l in range(L):
+        Lw = model.layers[l]
+        xh = rms_norm(h, Lw["attn_norm"], model.rms_eps)
+        q = (xh @ np.asarray(Lw["wq"], F64).T).reshape(1, n, Hq, hd)
+        k = (xh @ np.asarray(Lw["wk"], F64).T).reshape(1, n, Hkv, hd)
+        v = (xh @ np.asarray(Lw["wv"], F64).T).reshape(n, Hkv, hd)
+        q = rope_rotate_half(q, pos, model.rope_base)[0]
+        k = rope_rotate_half(k, pos, model.rope_base)[0]
+        kc[l], vc[l] = k, v
+        o = np.empty((n, Hq, hd))
+        for hq in range(Hq):
+            g = hq // group
+            sc = (q[:, hq, :] @ k[:, g, :].T) / math.sqrt(hd)
+            sc = np.where(causal, sc, -np.inf)
+            sc = sc - sc.max(axis=-1, keepdims=True)
+            p = np.exp(sc)
+            o[:, hq, :] = (p / p.sum(axis=-1, keepdims=True)) @ v[:, g, :]
+        h = h + o.reshape(n, Hq * hd) @ np.asarray(Lw["wo"], F64).T
+        hidden.append(h)
+        h = mlp_item(model, l, h[None])[0]
+        hidden.append(h)
+    return Prefill(k_cache=kc, v_cache=vc, hidden=np.stack(hidden))
+
+
+# --------------------------------------------------------------------------
 # Lemma 4.1 checker: does cosine closeness guarantee the same greedy token?
 # --------------------------------------------------------------------------
 @dataclass

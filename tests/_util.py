@@ -41,3 +41,24 @@ def oracle_model(inp) -> O.Model:
 
 def x0_np(inp) -> np.ndarray:
     return inp.x0.detach().double().cpu().numpy()
+
+
+def prefilled_inputs(name: str):
+    """The workload's seeded weights (with Wk / Wv) and the KV cache "from the
+    full model": the oracle's prefill over ctx + T seeded token embeddings, in
+    the workload's storage dtype; x0 = the last T embeddings.  Test input only."""
+    import dataclasses
+
+    from knapsack_layer_selection_b200 import workloads as W
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl)
+    ww = W.window_weights(wl)
+    inp = dataclasses.replace(inp, layers=[{**L, **w} for L, w in zip(inp.layers, ww)])
+    m = oracle_model(inp)
+    m = dataclasses.replace(m, layers=[m.layers[i] for i in range(len(m.layers))])
+    emb = W.sequence_embeddings(wl)
+    pf = O.prefill(m, emb.double().numpy())
+    dt = W.torch_dtype(wl)
+    kc = torch.from_numpy(pf.k_cache).to(dt)
+    vc = torch.from_numpy(pf.v_cache).to(dt)
+    return dataclasses.replace(inp, k_cache=kc, v_cache=vc, x0=emb[-wl.T:].contiguous())

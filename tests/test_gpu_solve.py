@@ -192,3 +192,25 @@ def test_distinct_state_solve_matches_oracle(name, mode, dedup):
     print(f"\n{name} {mode} dedup={dedup}: executed {int(s.out.exec_counts.sum())} states, "
           f"byte check rejected {int(s.out.dedup_rejected.sum())} fingerprint matches; {rep}")
     rep.assert_ok()
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_solve_on_the_full_model_cache_matches_oracle(name):
+    """The configurations' "KV cache from the full model": the cache is the
+    full model's own prefill over ctx + T tokens (oracle fp64, stored in the
+    workload's dtype), x0 the last T tokens' embeddings; full grid, taint rule."""
+    from tests._util import prefilled_inputs
+    inp = prefilled_inputs(name)
+    wl = inp.wl
+    t = wl.latencies()
+    w = O.quantize_weights(t, wl.n_bins)
+    g = inp.to("cuda")
+    solver = make_solver(wl, g, w=w, t=t)
+    solver.solve(g.x0)
+    res = gpu_result(solver)
+    orc = O.dp_solve(oracle_model(inp), x0_np(inp), wl.ctx, w, t, wl.gamma_max,
+                     per_cell=(wl.wdtype == "f32"))
+    rep = compare_solve(orc, res, w, VAL_TOL[wl.wdtype], wl.n_items, rows_val_gpu=res["rows"])
+    print(f"\n{name} on the full model's cache: best (b={orc.best_b}, gamma={orc.best_gamma}), "
+          f"min final value {np.nanmin(orc.values):.4f}; {rep}")
+    rep.assert_ok()

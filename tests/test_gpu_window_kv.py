@@ -81,9 +81,11 @@ def test_window_attention_sublayer_matches_oracle(name, E, ctx):
         og = O.apply_item(om, k, H.double().numpy(), ctx, kv="window")
         err = _branch_rel_err(out.double().cpu().numpy(), og, H.double().numpy())
         assert err < SUBLAYER_TOL[wl.wdtype], (k, err)
-        # the window reading differs from the cache reading (else nothing is tested)
+        # the window reading differs from the cache reading well beyond the
+        # tolerance (else nothing is tested); at long contexts the T window keys
+        # are a small share of the attention, so the gap is a few per cent
         oc = O.apply_item(om, k, H.double().numpy(), ctx, kv="cache")
-        assert _branch_rel_err(oc, og, H.double().numpy()) > 10 * SUBLAYER_TOL[wl.wdtype]
+        assert _branch_rel_err(oc, og, H.double().numpy()) > 3 * SUBLAYER_TOL[wl.wdtype]
         # a state's result depends only on its own rows
         assert torch.equal(out[1], out[2])
         assert torch.equal(out[1], one[0])
