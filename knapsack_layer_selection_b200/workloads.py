@@ -22,10 +22,11 @@ the paper uses are not available, so every tensor here is drawn at random:
 Draw order (one ``torch.Generator`` seeded with ``seed`` on ``device``): for each
 layer in order Wq, Wo, W_gate, W_up, W_down; then the K cache, the V cache, then
 x0.  Each tensor is drawn in fp32 and then rounded to the storage dtype.  Every
-workload that fits in host memory is drawn on the CPU generator (the 64 GB
-Qwen3-32B shape alone is drawn on the GPU's), so that a machine without a GPU
-can reproduce the inputs exactly; ``input_digest`` fingerprints a draw so that
-two machines can confirm they hold the same values.
+workload is drawn on the CPU generator, so that a machine without a GPU can
+reproduce the inputs exactly; ``input_digest`` fingerprints a draw so that two
+machines can confirm they hold the same values, and ``StreamedInputs`` holds
+only one layer at a time of a model too large for host memory (the 64 GB
+Qwen3-32B shape).
 """
 from __future__ import annotations
 
@@ -120,7 +121,7 @@ WORKLOADS: Dict[str, Workload] = {
     "qwen3_32b_16k": Workload("qwen3_32b_16k", n_layers=64, d_model=5120, n_q_heads=64,
                               n_kv_heads=8, head_dim=128, ffn=25600, rms_eps=1e-6,
                               rope_base=1e6, ctx=16384, T=8, wdtype="bf16", n_bins=1024,
-                              gamma_max=10, gen_device="cuda"),
+                              gamma_max=10, gen_device="cpu"),
 }
 
 # Order of the five workloads as the build's configuration list names them.
@@ -166,6 +167,35 @@ def _randn(shape, std, dtype, gen, device):
     return t.to(dtype)
 
 
+LAYER_KEYS = ("wq", "wo", "w_gate", "w_up", "w_down", "attn_norm", "mlp_norm")
+
+
+def _draw_layer(wl: Workload, gen, dev) -> Dict[str, torch.Tensor]:
+    """One layer's weights, drawn in the stated order."""
+    dt = torch_dtype(wl)
+    d, qd, F = wl.d_model, wl.q_dim, wl.ffn
+    layer = {
+        "wq": _randn((qd, d), LINEAR_STD, dt, gen, dev),
+        "wo": _randn((d, qd), LINEAR_STD, dt, gen, dev),
+        "w_gate": _randn((F, d), LINEAR_STD, dt, gen, dev),
+        "w_up": _randn((F, d), LINEAR_STD, dt, gen, dev),
+        "w_down": _randn((d, F), LINEAR_STD, dt, gen, dev),
+    }
+    layer["attn_norm"] = torch.ones(d, dtype=dt, device=dev)
+    layer["mlp_norm"] = torch.ones(d, dtype=dt, device=dev)
+    return layer
+
+
+def _draw_tail(wl: Workload, gen, dev):
+    """The K cache, the V cache and x0, drawn after every layer."""
+    dt = torch_dtype(wl)
+    kvshape = (wl.n_layers, wl.n_positions, wl.n_kv_heads, wl.head_dim)
+    k_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
+    v_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
+    x0 = _randn((wl.T, wl.d_model), 1.0, torch.float32, gen, dev)
+    return k_cache, v_cache, x0
+
+
 def make_inputs(wl: Workload, seed: int = 0, device: Optional[str] = None) -> Inputs:
     """Draw the workload's inputs (see the module docstring for the recipe)."""
     dev = device or wl.gen_device
@@ -173,26 +203,64 @@ def make_inputs(wl: Workload, seed: int = 0, device: Optional[str] = None) -> In
         raise RuntimeError(f"workload {wl.name} is drawn on CUDA, which is not available")
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
-    dt = torch_dtype(wl)
-    L = wl.n_layers
-    d, qd, F = wl.d_model, wl.q_dim, wl.ffn
-    layers = []
-    for _ in range(L):
-        layer = {
-            "wq": _randn((qd, d), LINEAR_STD, dt, gen, dev),
-            "wo": _randn((d, qd), LINEAR_STD, dt, gen, dev),
-            "w_gate": _randn((F, d), LINEAR_STD, dt, gen, dev),
-            "w_up": _randn((F, d), LINEAR_STD, dt, gen, dev),
-            "w_down": _randn((d, F), LINEAR_STD, dt, gen, dev),
-        }
-        layer["attn_norm"] = torch.ones(d, dtype=dt, device=dev)
-        layer["mlp_norm"] = torch.ones(d, dtype=dt, device=dev)
-        layers.append(layer)
-    kvshape = (L, wl.n_positions, wl.n_kv_heads, wl.head_dim)
-    k_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
-    v_cache = _randn(kvshape, kv_std(wl), dt, gen, dev)
-    x0 = _randn((wl.T, d), 1.0, torch.float32, gen, dev)
+    layers = [_draw_layer(wl, gen, dev) for _ in range(wl.n_layers)]
+    k_cache, v_cache, x0 = _draw_tail(wl, gen, dev)
     return Inputs(wl, layers, k_cache, v_cache, x0)
+
+
+class StreamedInputs:
+    """The CPU-generator inputs of a workload too large to hold at once.
+
+    The draw runs once in the stated order, keeping only the K/V cache and x0
+    and recording the generator's state at the start of every layer; a layer's
+    weights are drawn again from that state when asked for (``layers[l]``), so
+    they equal make_inputs(wl, seed, "cpu")'s.  ``digest`` equals input_digest
+    of that full draw, computed on the way.  ``to(device)`` places the whole
+    set on a device one layer at a time."""
+
+    def __init__(self, wl: Workload, seed: int = 0):
+        gen = torch.Generator(device="cpu")
+        gen.manual_seed(seed)
+        h = hashlib.sha256()
+        self.wl = wl
+        self._states = []
+        for _ in range(wl.n_layers):
+            self._states.append(gen.get_state())
+            layer = _draw_layer(wl, gen, "cpu")
+            for k in LAYER_KEYS:
+                _hash_update(h, layer[k])
+            del layer
+        self.k_cache, self.v_cache, self.x0 = _draw_tail(wl, gen, "cpu")
+        for l in range(wl.n_layers):
+            _hash_update(h, self.k_cache[l])
+        for l in range(wl.n_layers):
+            _hash_update(h, self.v_cache[l])
+        _hash_update(h, self.x0)
+        self.digest = h.hexdigest()
+        self.layers = _StreamedLayers(self)
+
+    def layer(self, l: int) -> Dict[str, torch.Tensor]:
+        gen = torch.Generator(device="cpu")
+        gen.set_state(self._states[l])
+        return _draw_layer(self.wl, gen, "cpu")
+
+    def to(self, device) -> Inputs:
+        layers = []
+        for l in range(self.wl.n_layers):
+            layers.append({k: v.to(device) for k, v in self.layer(l).items()})
+        return Inputs(self.wl, layers, self.k_cache.to(device), self.v_cache.to(device),
+                      self.x0.to(device))
+
+
+class _StreamedLayers:
+    def __init__(self, src: StreamedInputs):
+        self._src = src
+
+    def __len__(self):
+        return self._src.wl.n_layers
+
+    def __getitem__(self, l):
+        return self._src.layer(l)
 
 
 def window_weights(wl: Workload, seed: int = 2, device: Optional[str] = None
@@ -250,24 +318,24 @@ def random_states(shape: Sequence[int], seed: int, device: str = "cpu",
     return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32).to(dtype)
 
 
+def _hash_update(h, t: torch.Tensor) -> None:
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    h.update(t.numpy().tobytes())
+
+
 def input_digest(inp: Inputs) -> str:
     """SHA-256 of every input tensor's bytes, in draw order (weights layer by layer,
     then the K cache, the V cache and x0).  Two draws hold the same values iff
     their digests agree (up to hash collisions)."""
     h = hashlib.sha256()
-
-    def put(t: torch.Tensor):
-        t = t.detach().contiguous().cpu()
-        if t.dtype == torch.bfloat16:
-            t = t.view(torch.int16)
-        h.update(t.numpy().tobytes())
-
     for layer in inp.layers:
-        for k in ("wq", "wo", "w_gate", "w_up", "w_down", "attn_norm", "mlp_norm"):
-            put(layer[k])
+        for k in LAYER_KEYS:
+            _hash_update(h, layer[k])
     for l in range(inp.k_cache.shape[0]):
-        put(inp.k_cache[l])
+        _hash_update(h, inp.k_cache[l])
     for l in range(inp.v_cache.shape[0]):
-        put(inp.v_cache[l])
-    put(inp.x0)
+        _hash_update(h, inp.v_cache[l])
+    _hash_update(h, inp.x0)
     return h.hexdigest()

@@ -11,8 +11,9 @@ digest of the inputs so that the GPU machine can confirm it drew the same ones.
     python tests/golden/make_large_golden.py llama3_8b_8k
     python tests/golden/make_large_golden.py llama3_8b_32k --ctx 4096
 
-The 8B shape at 8k context takes about an hour on eight host cores (OpenBLAS
-fp64) and 30 GB of host memory.
+The 8B shape at 8k context takes about 25 minutes on eight host cores (OpenBLAS
+fp64) and 30 GB of host memory; the Qwen3-32B shape draws its layers one at a
+time (``StreamedInputs``) and needs about 15 GB.
 """
 from __future__ import annotations
 
@@ -48,7 +49,10 @@ def pack_sets(sets, n_items: int) -> np.ndarray:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("workload", choices=["llama3_8b_8k", "llama3_8b_32k", "small", "tiny"])
+    ap.add_argument("workload", choices=["llama3_8b_8k", "llama3_8b_32k", "qwen3_32b_16k", "small",
+                                         "tiny"])
+    ap.add_argument("--streamed", action="store_true",
+                    help="hold one layer of weights at a time (the 64 GB Qwen3-32B shape)")
     ap.add_argument("--ctx", type=int, default=None, help="context to solve at (default: the workload's)")
     ap.add_argument("--out", default=None)
     a = ap.parse_args()
@@ -56,8 +60,12 @@ def main():
     base = W.WORKLOADS[a.workload]
     wl = base.with_ctx(a.ctx) if a.ctx is not None else base
     t0 = time.time()
-    inp = W.make_inputs(base, device="cpu")        # the cache holds the workload's largest context
-    digest = W.input_digest(inp)
+    if a.streamed or a.workload == "qwen3_32b_16k":
+        inp = W.StreamedInputs(base)                # layers drawn again when the oracle reads them
+        digest = inp.digest
+    else:
+        inp = W.make_inputs(base, device="cpu")    # the cache holds the workload's largest context
+        digest = W.input_digest(inp)
     print(f"{a.workload}: inputs drawn and hashed in {time.time() - t0:.0f} s, sha256 {digest}",
           flush=True)
 

@@ -1,7 +1,7 @@
 """The seeded synthetic inputs follow their stated recipe: shapes, dtypes, draw
 order, spreads and determinism; the latency models give each workload its
-stated item weights and budget grid.  CPU only (the large shapes are drawn on
-the GPU, so only their latency side is checked here)."""
+stated item weights and budget grid.  CPU only (the large shapes are checked
+through their latency side; their draw uses the same code as the small shapes)."""
 import math
 
 import pytest
@@ -90,3 +90,24 @@ def test_lm_head_and_random_states():
     assert torch.equal(h, W.lm_head(wl)) and not torch.equal(h, W.lm_head(wl, seed=2))
     s = W.random_states((3, 4, 8), 5)
     assert torch.equal(s, W.random_states((3, 4, 8), 5)) and s.dtype == torch.float32
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_streamed_inputs_equal_the_full_draw(name):
+    """StreamedInputs (one layer held at a time, each redrawn from its recorded
+    generator state) gives the same values and the same digest as make_inputs."""
+    wl = W.WORKLOADS[name]
+    full = W.make_inputs(wl)
+    st = W.StreamedInputs(wl)
+    assert st.digest == W.input_digest(full)
+    for l in (wl.n_layers - 1, 0, 1):               # any order: each layer from its own state
+        for k in W.LAYER_KEYS:
+            assert torch.equal(st.layers[l][k], full.layers[l][k]), (l, k)
+    assert torch.equal(st.k_cache, full.k_cache) and torch.equal(st.v_cache, full.v_cache)
+    assert torch.equal(st.x0, full.x0)
+    # a different seed changes the digest
+    assert W.StreamedInputs(wl, seed=1).digest != st.digest
+
+
+def test_every_workload_is_drawn_on_the_cpu_generator():
+    assert all(wl.gen_device == "cpu" for wl in W.WORKLOADS.values())
