@@ -128,6 +128,109 @@ __device__ __forceinline__ int tile_group(const GemmParams& p, int tm, int& loca
   return g;
 }
 
+// The fused epilogue of one accumulator row: this thread's TMEM lane holds row
+// `row` of the tile, 256 columns from tbase, for output columns tn * 256 (tn * 128
+// for SwiGLU).  Stores nothing for a row past M (but still reads TMEM, a
+// warp-collective operation).
+template <int EPI>
+__device__ __forceinline__ void epilogue_row(const GemmParams& p, void* g_out, const float* g_resid,
+                                             const float2* g_rope, int row, bool live, int tn,
+                                             uint32_t tbase) {
+  float v[32], u[32];
+  if (EPI == EPI_RESID_F32 || EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
+    const int n0 = tn * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      tmem_ld32(tbase + c * 32, v);
+      tmem_wait_ld();
+      if (!live) continue;
+      const long long off = (long long)row * p.N_out + n0 + c * 32;
+      if (EPI == EPI_STORE_BF16) {
+        store_bf16x32((__nv_bfloat16*)g_out + off, v);
+      } else {
+        float4* o = reinterpret_cast<float4*>((float*)g_out + off);
+        if (EPI == EPI_RESID_F32) {
+          const float4* rr = reinterpret_cast<const float4*>(g_resid + off);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 x = rr[j];
+            o[j] = make_float4(v[4 * j] + x.x, v[4 * j + 1] + x.y, v[4 * j + 2] + x.z,
+                               v[4 * j + 3] + x.w);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+    }
+  } else if (EPI == EPI_ROWMAX) {
+    // top-2 of scale * acc + bias over this tile's 256 columns of the row
+    const int n0 = tn * BN;
+    float v1 = -INFINITY, v2 = -INFINITY;
+    int i1 = -1;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      tmem_ld32(tbase + c * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int col = n0 + c * 32 + j;
+        const float x = p.rowmax.scale * v[j] + (p.rowmax.col_bias ? p.rowmax.col_bias[col] : 0.f);
+        if (x > v1) {
+          v2 = v1;
+          v1 = x;
+          i1 = col;
+        } else if (x > v2) {
+          v2 = x;
+        }
+      }
+    }
+    if (live)
+      reinterpret_cast<float4*>(g_out)[(long long)row * p.tiles_n + tn] =
+          make_float4(v1, __int_as_float(i1), v2, 0.f);
+  } else if (EPI == EPI_SWIGLU_BF16) {
+    // columns 0..127: gate, 128..255: up, for output columns tn*128 ..
+    const int n0 = tn * (BN / 2);
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+      tmem_ld32(tbase + c * 32, v);
+      tmem_ld32(tbase + BN / 2 + c * 32, u);
+      tmem_wait_ld();
+      if (!live) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] / (1.0f + __expf(-v[j])) * u[j];
+      store_bf16x32((__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + c * 32, v);
+    }
+  } else if (EPI == EPI_ROPE_BF16) {
+    // rotate-half RoPE inside each head of this tile: column j pairs with j + hd/2
+    const int half = p.head_dim / 2;
+    const int tok = row % p.T;
+    const float2* cs = g_rope + (long long)tok * half;
+    const int n0 = tn * BN;
+#pragma unroll 1
+    for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
+#pragma unroll 1
+      for (int c = 0; c < half; c += 32) {
+        tmem_ld32(tbase + h0 + c, v);
+        tmem_ld32(tbase + h0 + half + c, u);
+        tmem_wait_ld();
+        if (!live) continue;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float2 r = cs[c + j];
+          const float x1 = v[j], x2 = u[j];
+          v[j] = x1 * r.x - x2 * r.y;
+          u[j] = x2 * r.x + x1 * r.y;
+        }
+        __nv_bfloat16* o = (__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + h0 + c;
+        store_bf16x32(o, v);
+        store_bf16x32(o + half, u);
+      }
+    }
+  }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA1,
@@ -274,99 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int row = m0 + q * 32 + lane;
       const bool live = row < (gi == 0 ? m_live0 : gr.M);
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      float v[32], u[32];
-      if (EPI == EPI_RESID_F32 || EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
-        const int n0 = tn * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_ld32(tbase + c * 32, v);
-          tmem_wait_ld();
-          if (!live) continue;
-          const long long off = (long long)row * p.N_out + n0 + c * 32;
-          if (EPI == EPI_STORE_BF16) {
-            store_bf16x32((__nv_bfloat16*)g_out + off, v);
-          } else {
-            float4* o = reinterpret_cast<float4*>((float*)g_out + off);
-            if (EPI == EPI_RESID_F32) {
-              const float4* rr = reinterpret_cast<const float4*>(g_resid + off);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 x = rr[j];
-                o[j] = make_float4(v[4 * j] + x.x, v[4 * j + 1] + x.y, v[4 * j + 2] + x.z,
-                                   v[4 * j + 3] + x.w);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            }
-          }
-        }
-      } else if (EPI == EPI_ROWMAX) {
-        // top-2 of scale * acc + bias over this tile's 256 columns of the row
-        const int n0 = tn * BN;
-        float v1 = -INFINITY, v2 = -INFINITY;
-        int i1 = -1;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_ld32(tbase + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = n0 + c * 32 + j;
-            const float x = p.rowmax.scale * v[j] + (p.rowmax.col_bias ? p.rowmax.col_bias[col] : 0.f);
-            if (x > v1) {
-              v2 = v1;
-              v1 = x;
-              i1 = col;
-            } else if (x > v2) {
-              v2 = x;
-            }
-          }
-        }
-        if (live)
-          reinterpret_cast<float4*>(g_out)[(long long)row * p.tiles_n + tn] =
-              make_float4(v1, __int_as_float(i1), v2, 0.f);
-      } else if (EPI == EPI_SWIGLU_BF16) {
-        // columns 0..127: gate, 128..255: up, for output columns tn*128 ..
-        const int n0 = tn * (BN / 2);
-#pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
-          tmem_ld32(tbase + c * 32, v);
-          tmem_ld32(tbase + BN / 2 + c * 32, u);
-          tmem_wait_ld();
-          if (!live) continue;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = v[j] / (1.0f + __expf(-v[j])) * u[j];
-          store_bf16x32((__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + c * 32, v);
-        }
-      } else if (EPI == EPI_ROPE_BF16) {
-        // rotate-half RoPE inside each head of this tile: column j pairs with j + hd/2
-        const int half = p.head_dim / 2;
-        const int tok = row % p.T;
-        const float2* cs = g_rope + (long long)tok * half;
-        const int n0 = tn * BN;
-#pragma unroll 1
-        for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
-#pragma unroll 1
-          for (int c = 0; c < half; c += 32) {
-            tmem_ld32(tbase + h0 + c, v);
-            tmem_ld32(tbase + h0 + half + c, u);
-            tmem_wait_ld();
-            if (!live) continue;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 r = cs[c + j];
-              const float x1 = v[j], x2 = u[j];
-              v[j] = x1 * r.x - x2 * r.y;
-              u[j] = x2 * r.x + x1 * r.y;
-            }
-            __nv_bfloat16* o = (__nv_bfloat16*)g_out + (long long)row * p.N_out + n0 + h0 + c;
-            store_bf16x32(o, v);
-            store_bf16x32(o + half, u);
-          }
-        }
-      }
+      epilogue_row<EPI>(p, g_out, g_resid, g_rope, row, live, tn, tbase);
       tc_fence_before();
       mbar_arrive(smem_u32(&tail->tempty[acc]));
     }
@@ -377,6 +388,194 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- the CTA-pair GEMM
+// The same product and epilogues on 256 x 256 tiles computed by a pair of CTAs
+// on two SMs (a 2-CTA cluster) with the pair MMA (tcgen05.mma.cta_group::2, M =
+// 256): each CTA loads its own 128 rows of A and its half of the tile's 256
+// weight rows, so per SM a k-step moves 32 KB instead of 48 KB for the same
+// tensor work, and six stages fit where four did -- half again as much time to
+// hide each stage's load behind the MMAs.  The leader CTA (rank 0) arms each
+// stage's barrier for both CTAs' bytes and issues the MMAs; its commits arrive
+// on both CTAs' barriers; both CTAs' epilogues read their own 128 TMEM rows and
+// release the accumulator on the leader's barrier.  Every wait is bounded, and
+// a cluster barrier at the end keeps either CTA from leaving while the other may
+// still touch its shared memory.  A tile's arithmetic is the same fixed-order
+// sum over K as in tc_gemm_kernel.
+constexpr int BM2 = 256;
+constexpr int STAGES2 = 6;
+constexpr int A2_BYTES = 128 * BK * 2;       // this CTA's 128 rows of A: 16 KB
+constexpr int B2_BYTES = 128 * BK * 2;       // this CTA's half of the 256 weight rows: 16 KB
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t IDESC2 = idesc_bf16_f32(BM2, BN);
+
+struct SharedTail2 {
+  uint64_t full[STAGES2];   // leader: both CTAs' bytes of a stage have landed
+  uint64_t empty[STAGES2];  // each CTA: the pair MMAs reading a stage are done
+  uint64_t tfull[2];        // each CTA: an accumulator is complete
+  uint64_t tempty[2];       // leader: both CTAs' epilogues have read an accumulator
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SharedTail2) <= 256, "barrier block");
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmA2,
+                        const __grid_constant__ CUtensorMap tmA3,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB2, const GemmParams p_in) {
+  GemmParams p = p_in;
+  int m_live0 = p_in.grp[0].M;
+  if (p.dyn_cells) {
+    const long long live = (long long)(*p.dyn_cells) * p.T;
+    m_live0 = (int)(live < m_live0 ? live : m_live0);
+    p.tiles_m = (m_live0 + BM2 - 1) / BM2;
+    if (p.group_m > p.tiles_m) p.group_m = p.tiles_m > 0 ? p.tiles_m : 1;
+  }
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  SharedTail2* tail = reinterpret_cast<SharedTail2*>(smem + STAGES2 * STAGE2_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), n_pairs = (int)(gridDim.x >> 1);
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  const int KB = p.K / BK;
+  volatile int* abort = &tail->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(smem_u32(&tail->full[s]), 1);
+      mbar_init(smem_u32(&tail->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tail->tfull[a]), 1);
+      mbar_init(smem_u32(&tail->tempty[a]), 2 * 128);   // every epilogue thread of both CTAs
+    }
+    mbar_init(smem_u32(&tail->drain), 1);
+    tail->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    if (p.n_groups > 1) prefetch_tmap(&tmA1);
+    if (p.n_groups > 2) prefetch_tmap(&tmA2);
+    if (p.n_groups > 3) prefetch_tmap(&tmA3);
+    prefetch_tmap(&tmB);
+    if (EPI == EPI_SWIGLU_BF16) prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&tail->tmem_base), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();           // the peer's barriers exist before any remote arrival
+  const uint32_t tmem_base = tail->tmem_base;
+  const uint32_t full_leader = cluster_addr(smem_u32(&tail->full[0]), 0);
+  const uint32_t tempty_leader = cluster_addr(smem_u32(&tail->tempty[0]), 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        int tmg, tn, tm;
+        tile_coords(p, t, tmg, tn);
+        const int grp = tile_group(p, tmg, tm);
+        const CUtensorMap* am = grp == 0 ? &tmA : grp == 1 ? &tmA1 : grp == 2 ? &tmA2 : &tmA3;
+        const int m0 = tm * BM2 + (int)rank * 128;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES2;
+          const uint32_t r = (uint32_t)(it / STAGES2);
+          if (!mbar_wait(smem_u32(&tail->empty[s]), (r & 1u) ^ 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_leader + 8u * (uint32_t)s;
+          if (leader) mbar_arrive_expect_tx(smem_u32(&tail->full[s]), 2 * STAGE2_BYTES);
+          const uint32_t a_dst = smem_u32(smem + s * STAGE2_BYTES);
+          const uint32_t b_dst = a_dst + A2_BYTES;
+          tma_load_2d_pair(a_dst, am, kb * BK, m0, fb);
+          if (EPI == EPI_SWIGLU_BF16)   // gate rows in the leader, up rows in the peer
+            tma_load_2d_pair(b_dst, leader ? &tmB : &tmB2, kb * BK, tn * (BN / 2), fb);
+          else
+            tma_load_2d_pair(b_dst, &tmB, kb * BK, tn * BN + (int)rank * 128, fb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer (leader)
+    if (lane == 0 && leader) {
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++i) {
+        const int acc = i & 1;
+        const uint32_t ar = (uint32_t)(i >> 1);
+        if (!mbar_wait(smem_u32(&tail->tempty[acc]), (ar & 1u) ^ 1u, abort, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES2;
+          const uint32_t r = (uint32_t)(it / STAGES2);
+          if (!mbar_wait(smem_u32(&tail->full[s]), r & 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE2_BYTES);
+          const uint64_t a_desc = desc_kmajor_sw128(a_addr);
+          const uint64_t b_desc = desc_kmajor_sw128(a_addr + A2_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, IDESC2, (kb | k) != 0);
+          mma_commit_pair_both(smem_u32(&tail->empty[s]));
+        }
+        if (!ok) break;
+        mma_commit_pair_both(smem_u32(&tail->tfull[acc]));
+      }
+      // every pair MMA issued above retires before TMEM is released
+      mma_commit_pair_self(smem_u32(&tail->drain));
+      mbar_wait_drain(smem_u32(&tail->drain), 0, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
+    const int q = warp & 3;
+    int i = 0;
+    for (int t = pair; t < n_tiles; t += n_pairs, ++i) {
+      const int acc = i & 1;
+      const uint32_t ar = (uint32_t)(i >> 1);
+      const bool got = mbar_wait(smem_u32(&tail->tfull[acc]), ar & 1u, abort, p.status);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      int tmg, tn, tm;
+      tile_coords(p, t, tmg, tn);
+      const int gi = tile_group(p, tmg, tm);
+      const GemmGroupDev& gr = p_in.grp[gi];
+      const int row = tm * BM2 + (int)rank * 128 + q * 32 + lane;
+      const bool live = row < (gi == 0 ? m_live0 : gr.M);
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      epilogue_row<EPI>(p, gr.out, gr.resid, gr.rope_cs, row, live, tn, tbase);
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();           // neither CTA leaves while its peer may still reach it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -418,6 +617,38 @@ ks_status launch(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& 
   const int n_tiles = gp.tiles_m * gp.tiles_n;
   const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
   k<<<grid, THREADS, SMEM_BYTES, st>>>(a[0], a[1], a[2], a[3], b, b2, gp);
+  KS_LAUNCH_CHECK();
+  return KS_OK;
+}
+
+// Pairs of CTAs that can be resident at once (a persistent grid of that many pairs).
+template <int EPI>
+ks_status launch_pair(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& b2,
+                      const GemmParams& gp, cudaStream_t st) {
+  static std::atomic<unsigned long long> attr_set{0};
+  static int max_pairs = 0;
+  auto k = tc_gemm_pair_kernel<EPI>;
+  KS_TRY(once_per_device(attr_set, [&]() -> ks_status {
+    KS_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * sm_count());
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 2;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n < 1) n = sm_count() / 2;
+    max_pairs = n;
+    return KS_OK;
+  }));
+  const int n_tiles = gp.tiles_m * gp.tiles_n;
+  const int pairs = n_tiles < max_pairs ? n_tiles : max_pairs;
+  k<<<2 * pairs, THREADS, SMEM2_BYTES, st>>>(a[0], a[1], a[2], a[3], b, b2, gp);
   KS_LAUNCH_CHECK();
   return KS_OK;
 }
@@ -466,6 +697,10 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
   GemmParams gp{};
   CUtensorMap ta[kGemmMaxGroups], tb, tb2;
   int tiles_m = 0, n_live = 0;
+  // CTA pairs for every product but the row-maximum scan; each CTA then loads
+  // 128-row boxes of A and of the weights
+  const bool pair = epi != EPI_ROWMAX;
+  const int bm = pair ? BM2 : BM;
   for (int g = 0; g < n_groups; ++g) {
     const GemmGroupArg& a = groups[g];
     if (a.M <= 0) continue;                     // an empty group takes no tiles
@@ -475,7 +710,7 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
       return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: resid is NULL");
     KS_TRY(make_tmap_2d(&ta[n_live], a.A, a.M, K, K, BK, BM));
     gp.grp[n_live] = GemmGroupDev{a.out, a.resid, a.rope_cs, a.M, tiles_m};
-    tiles_m += (a.M + BM - 1) / BM;
+    tiles_m += (a.M + bm - 1) / bm;
     ++n_live;
   }
   if (n_live == 0) return KS_OK;
@@ -484,7 +719,7 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
     KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN / 2));
     KS_TRY(make_tmap_2d(&tb2, B2, N, K, K, BK, BN / 2));
   } else {
-    KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, BN));
+    KS_TRY(make_tmap_2d(&tb, B, N, K, K, BK, pair ? BN / 2 : BN));
     tb2 = tb;
   }
   gp.n_groups = n_live;
@@ -503,7 +738,7 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
   // the second).  The walk changes only which CTA computes a tile and when, never
   // a tile's arithmetic.
   {
-    const long long a_tile = (long long)BM * K * 2;
+    const long long a_tile = (long long)bm * K * 2;
     const long long b_tile = (long long)BN * K * 2;
     long long g = (32ll << 20) / a_tile;
     if (g < 8) g = 8;
@@ -522,11 +757,11 @@ ks_status tc_gemm_groups(const GemmGroupArg* groups, int n_groups, const void* B
   gp.dyn_cells = dyn_cells;
   gp.rowmax = rowmax;
   switch (epi) {
-    case EPI_RESID_F32: return launch<EPI_RESID_F32>(ta, tb, tb2, gp, st);
-    case EPI_ROPE_BF16: return launch<EPI_ROPE_BF16>(ta, tb, tb2, gp, st);
-    case EPI_SWIGLU_BF16: return launch<EPI_SWIGLU_BF16>(ta, tb, tb2, gp, st);
-    case EPI_STORE_BF16: return launch<EPI_STORE_BF16>(ta, tb, tb2, gp, st);
-    case EPI_STORE_F32: return launch<EPI_STORE_F32>(ta, tb, tb2, gp, st);
+    case EPI_RESID_F32: return launch_pair<EPI_RESID_F32>(ta, tb, tb2, gp, st);
+    case EPI_ROPE_BF16: return launch_pair<EPI_ROPE_BF16>(ta, tb, tb2, gp, st);
+    case EPI_SWIGLU_BF16: return launch_pair<EPI_SWIGLU_BF16>(ta, tb, tb2, gp, st);
+    case EPI_STORE_BF16: return launch_pair<EPI_STORE_BF16>(ta, tb, tb2, gp, st);
+    case EPI_STORE_F32: return launch_pair<EPI_STORE_F32>(ta, tb, tb2, gp, st);
     case EPI_ROWMAX: return launch<EPI_ROWMAX>(ta, tb, tb2, gp, st);
   }
   return fail(KS_ERR_INVALID_ARG, "tensor-core GEMM: unknown epilogue");
