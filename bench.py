@@ -434,6 +434,45 @@ def run_ours(args, rank, world, local):
                   "identical_to_dense": same}
     del dd
 
+    # ---- the DP re-solved at three contexts (the cache covers them): three separate
+    # solves against one pass that shares every GEMM's weight reads; identical results
+    ctxs = [wl.ctx // 4, wl.ctx // 2, wl.ctx]
+    m = B.model_desc(wl.n_layers, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                     wl.rms_eps, wl.rope_base, wl.wdtype)
+    prm = B.params(wl.gamma_max, wl.n_bins)
+    sep = [B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, c, wl.T, wl.with_ctx(c).latencies(),
+                    prm, keep_bp=False, keep_tpt=False, keep_ref=False) for c in ctxs]
+    one = B.SolverContexts(m, inp.layers, [(inp.k_cache, inp.v_cache, c) for c in ctxs], wl.T,
+                           [wl.with_ctx(c).latencies() for c in ctxs], prm, keep_bp=False,
+                           keep_tpt=False, keep_ref=False)
+    for _ in range(2):
+        for sv in sep:
+            sv.solve(x0)
+        one.solve([x0] * len(ctxs))
+    torch.cuda.synchronize()
+    reps = max(1, min(args.steps, 3))
+    e6, e7, e8 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    barrier(world)
+    e6.record(stream)
+    for _ in range(reps):
+        for sv in sep:
+            sv.solve(x0)
+    e7.record(stream)
+    for _ in range(reps):
+        one.solve([x0] * len(ctxs))
+    e8.record(stream)
+    torch.cuda.synchronize()
+    for sv in sep:
+        sv.check_status()
+    one.check_status()
+    same_ctx = all(torch.equal(a.out.values, b.values) and torch.equal(a.out.sets, b.sets) and
+                   torch.equal(a.out.best, b.best) for a, b in zip(sep, one.outs))
+    contexts_line = {"contexts": ctxs, "cells": one.C,
+                     "separate_ms": max_over_ranks(e6.elapsed_time(e7) / reps, world),
+                     "one_pass_ms": max_over_ranks(e7.elapsed_time(e8) / reps, world),
+                     "identical": same_ctx}
+    del sep, one
+
     cpu = None
     if rank == 0 and world == 1:
         v, desc, threads, _ = oracle_sample(wl, inp, args.cpu_seconds)
@@ -463,6 +502,7 @@ def run_ours(args, rank, world, local):
                         "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "dedup": dedup_line,
+                "contexts": contexts_line,
                 "gpu_launches": launches * args.steps,
                 "kernels": {s["name"]: {"launches_per_step": s["launches"] // args.steps,
                                         "ms_per_step": s["total_ms"] / args.steps,
