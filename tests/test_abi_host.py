@@ -337,3 +337,16 @@ def test_solve_contexts_checks_before_any_launch(lib):
     one = [B.workspace_size(m, c, 4) for c in (9, 33)]
     assert sum(one) <= size.value <= sum(one) + 512
     assert lib.ks_workspace_size_contexts(ctypes.byref(m), 5, cells, 4, ctypes.byref(size)) == 1
+
+
+def test_library_leaves_none_of_its_own_symbols_undefined(lib):
+    """Every function of the library's namespace that one file calls is defined
+    (with external linkage) in another: nothing of its own is left for dlopen."""
+    import shutil
+    import subprocess
+    if shutil.which("nm") is None:
+        pytest.skip("nm is not available")
+    out = subprocess.run(["nm", "-D", "--undefined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    own = [l for l in out.splitlines() if "_ZN2ks" in l or " ks_" in l]
+    assert own == [], own
