@@ -206,6 +206,27 @@ def solver_for(wl, inp, keep=False, dedup=False):
                     keep_bp=keep, keep_cos=False, keep_tpt=keep, keep_ref=keep)
 
 
+def select_bytes(wl, C: int, w, bp: torch.Tensor, keep_ref: bool) -> float:
+    """Algorithmic DRAM bytes of one solve's select launches, from the solve's own
+    decisions (bp, [items x C]).  Per item k: reads of the reference slot, of every
+    cell's skip candidate and of the C - w_k execute candidates (the target is the
+    reference slot's output); writes of the reference slot, of the cells whose
+    execute candidate won (the others keep their state in place), of the
+    reference-state copy when kept, and of every slot's normalised operand of the
+    next item."""
+    cell = wl.T * wl.d_model
+    xb = 2 if wl.wdtype == "bf16" else 4
+    takes = bp.to(torch.int64).sum(dim=1).tolist()
+    n = len(w)
+    total = 0.0
+    for k, wk in enumerate(w):
+        total += (1 + C + (C - wk)) * cell * 4.0
+        total += (1 + takes[k] + (1 if keep_ref else 0)) * cell * 4.0
+        if k + 1 < n:
+            total += (C + 1) * cell * xb
+    return total
+
+
 def oracle_sample(wl, inp, seconds: float):
     """Time the oracle (as it stands) on a bounded sample of the workload.
 
@@ -428,6 +449,22 @@ def run_ours(args, rank, world, local):
     same = bool(torch.equal(dd.out.values, solver.out.values) and
                 torch.equal(dd.out.sets, solver.out.sets) and
                 torch.equal(dd.out.best, solver.out.best))
+    # ---- the select's own roofline: its algorithmic bytes counted from one solve's
+    # backpointers (the timed solves are the same computation on the same inputs)
+    chk = solver_for(wl, inp, keep=True)
+    chk.solve(x0)
+    torch.cuda.synchronize()
+    chk.check_status()
+    sel_bytes = select_bytes(wl, C, solver.w, chk.out.bp, keep_ref=False)
+    del chk
+    sel_ms = kinds["select_bp"]["total_ms"] / args.steps if "select_bp" in kinds else None
+    select_line = None
+    if sel_ms:
+        sel_gbs = sel_bytes / (sel_ms / 1000.0) / 1e9
+        select_line = {"kernel": "select_bp", "bound": "hbm", "bytes_per_step": sel_bytes,
+                       "ms_per_step": sel_ms, "achieved": sel_gbs, "peak": peaks["hbm_gbs"],
+                       "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
+                       "peak_source": f"{peak_src} hbm copy"}
     dedup_line = {"solve_ms": dd_ms, "value": job_value(units, dd_ms, world), "unit": UNIT,
                   "states_executed": ran, "states_dense": dense_cells,
                   "executed_fraction": ran / dense_cells, "speedup_vs_dense": ms / dd_ms,
@@ -501,6 +538,7 @@ def run_ours(args, rank, world, local):
                 "e2e": {"value": job_value(units, e2e_ms, world), "unit": UNIT,
                         "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
+                "select_roofline": select_line,
                 "dedup": dedup_line,
                 "contexts": contexts_line,
                 "gpu_launches": launches * args.steps,

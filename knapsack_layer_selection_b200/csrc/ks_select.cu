@@ -299,26 +299,34 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_fused_kernel(
   float4* rdst = (is_ref && ref_out) ? (float4*)ref_out : nullptr;
   TX* xdst = g_next ? xh_next + slot * cell : nullptr;
   const long long n4 = cell / 4;
+  constexpr int U2 = 4;   // copy pass: four loads in flight per thread (its reads hit L2 in part)
+  // float4 i of the cell is column j4 of token t (i = t * d4 + j4); stepping i by
+  // the block size moves (t, j4) by (qB, rB), so the loop divides nothing
+  const int B = blockDim.x;
+  const int qB = B / d4, rB = B - qB * d4;
+  int t0 = (int)threadIdx.x / d4, j0 = (int)threadIdx.x - t0 * d4;
   Hash2 hh;
-  for (long long i0 = threadIdx.x; i0 < n4; i0 += (long long)blockDim.x * U) {
-    float4 vv[U];
+  for (long long i0 = threadIdx.x; i0 < n4; i0 += (long long)B * U2) {
+    float4 vv[U2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long i = i0 + (long long)u * blockDim.x;
+    for (int u = 0; u < U2; ++u) {
+      const long long i = i0 + (long long)u * B;
       if (i < n4) vv[u] = src[i];
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long i = i0 + (long long)u * blockDim.x;
+    for (int u = 0; u < U2; ++u) {
+      const long long i = i0 + (long long)u * B;
       if (i >= n4) break;
       const float4 v = vv[u];
       if (dst) dst[i] = v;
       if (rdst) rdst[i] = v;
       if (hash_cur) hh.add4(v, (uint32_t)(i * 4));
-      if (xdst) {
-        const int t = (int)(i / d4);
-        const int j = (int)(i - (long long)t * d4) * 4;
-        store_norm4(xdst + i * 4, v, inv[t], g_next + j);
+      if (xdst) store_norm4(xdst + i * 4, v, inv[t0], g_next + 4 * j0);
+      t0 += qB;
+      j0 += rB;
+      if (j0 >= d4) {
+        j0 -= d4;
+        ++t0;
       }
     }
   }
@@ -376,15 +384,23 @@ __global__ void __launch_bounds__(kSelectThreads) init_states_kernel(
   float4* dst = (float4*)(states + slot * cell);
   float4* rdst = (slot == 0 && ref_out) ? (float4*)ref_out : nullptr;
   TX* xdst = xh + slot * cell;
+  // (t, j4) of float4 i = t * d4 + j4, stepped with i
+  const int B = blockDim.x;
+  const int qB = B / d4, rB = B - qB * d4;
+  int t = (int)threadIdx.x / d4, j4 = (int)threadIdx.x - t * d4;
   Hash2 hh;
-  for (long long i = threadIdx.x; i < cell / 4; i += blockDim.x) {
+  for (long long i = threadIdx.x; i < cell / 4; i += B) {
     const float4 v = src[i];
     dst[i] = v;
     if (rdst) rdst[i] = v;
     if (hash_out) hh.add4(v, (uint32_t)(i * 4));
-    const int t = (int)(i / d4);
-    const int j = (int)(i - (long long)t * d4) * 4;
-    store_norm4(xdst + i * 4, v, inv_s[t], g + j);
+    store_norm4(xdst + i * 4, v, inv_s[t], g + 4 * j4);
+    t += qB;
+    j4 += rB;
+    if (j4 >= d4) {
+      j4 -= d4;
+      ++t;
+    }
   }
   if (hash_out) block_hash_store(hh, hash_sh, hash_out + slot);
 }
