@@ -65,13 +65,17 @@ def solve_case(full, repeat):
     m = B.model_desc(2, wl.d_model, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
                      wl.rms_eps, wl.rope_base, wl.wdtype)
     s = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, t,
-                 B.params(wl.gamma_max, full.n_bins), w=w, keep_bp=False, keep_tpt=False,
+                 B.params(wl.gamma_max, full.n_bins), w=w, keep_bp=True, keep_tpt=False,
                  keep_ref=False)
     for _ in range(repeat):
         s.solve(inp.x0)
     torch.cuda.synchronize()
     s.check_status()
-    print(f"{full.name} solve: 2 layers, {s.C} cells x {wl.T} tokens, {repeat} solve(s) ok")
+    # per item: the cells whose execute candidate won (the select writes only
+    # those states; the others stay in place)
+    takes = s.out.bp.to(torch.int64).sum(dim=1).tolist()
+    print(f"{full.name} solve: 2 layers, {s.C} cells x {wl.T} tokens, {repeat} solve(s) ok; "
+          f"item weights {w}, execute wins per item {takes}")
 
 
 if __name__ == "__main__":

@@ -216,19 +216,24 @@ class StreamedInputs:
     weights are drawn again from that state when asked for (``layers[l]``), so
     they equal make_inputs(wl, seed, "cpu")'s.  ``digest`` equals input_digest
     of that full draw, computed on the way.  ``to(device)`` places the whole
-    set on a device one layer at a time."""
+    set on a device one layer at a time; with ``device`` given, each layer is
+    copied there as it is drawn, and ``to(device)`` then draws nothing again."""
 
-    def __init__(self, wl: Workload, seed: int = 0):
+    def __init__(self, wl: Workload, seed: int = 0, device: Optional[str] = None):
         gen = torch.Generator(device="cpu")
         gen.manual_seed(seed)
         h = hashlib.sha256()
         self.wl = wl
         self._states = []
+        self._device = device
+        self._dev_layers = []
         for _ in range(wl.n_layers):
             self._states.append(gen.get_state())
             layer = _draw_layer(wl, gen, "cpu")
             for k in LAYER_KEYS:
                 _hash_update(h, layer[k])
+            if device is not None:
+                self._dev_layers.append({k: v.to(device) for k, v in layer.items()})
             del layer
         self.k_cache, self.v_cache, self.x0 = _draw_tail(wl, gen, "cpu")
         for l in range(wl.n_layers):
@@ -245,9 +250,11 @@ class StreamedInputs:
         return _draw_layer(self.wl, gen, "cpu")
 
     def to(self, device) -> Inputs:
-        layers = []
-        for l in range(self.wl.n_layers):
-            layers.append({k: v.to(device) for k, v in self.layer(l).items()})
+        if self._device is not None and torch.device(device) == torch.device(self._device):
+            layers = self._dev_layers
+        else:
+            layers = [{k: v.to(device) for k, v in self.layer(l).items()}
+                      for l in range(self.wl.n_layers)]
         return Inputs(self.wl, layers, self.k_cache.to(device), self.v_cache.to(device),
                       self.x0.to(device))
 

@@ -95,3 +95,23 @@ def test_attention_is_deterministic_at_long_context():
             first = out
         else:
             assert torch.equal(first, out)
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+def test_attention_with_a_maximum_that_keeps_growing(hd):
+    """Keys whose norm grows with position: the row maximum rises block after
+    block, so the reference moves often (O rescaled in place, and each softmax
+    group's own row sum brought to the new reference) in both groups' blocks."""
+    R, T, Hq, Hkv, ctx = 256, 16, 8, 2, 2000
+    q, k, v = _case(R, T, Hq, Hkv, hd, ctx, seed=33)
+    ramp = 1.0 + torch.arange(k.shape[0], device="cuda", dtype=torch.float32) / 256.0
+    k = (k.float() * ramp[:, None, None]).to(torch.bfloat16)
+    out = torch.empty(R, Hq, hd, device="cuda", dtype=torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    B.attention_bf16(q, k, v, T, ctx, out, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = _reference(q, k, v, T, ctx)
+    rel = ((out.float() - ref).norm() / ref.norm()).item()
+    worst = (out.float() - ref).abs().max().item()
+    assert rel < 1e-2 and worst < 5e-2 * ref.abs().max().item(), (rel, worst)

@@ -109,5 +109,20 @@ def test_streamed_inputs_equal_the_full_draw(name):
     assert W.StreamedInputs(wl, seed=1).digest != st.digest
 
 
+def test_streamed_inputs_kept_on_a_device_need_no_second_draw(monkeypatch):
+    """With a device given, the layers are copied there while the digest is taken,
+    and to(device) hands those copies back without drawing again."""
+    wl = W.WORKLOADS["tiny"]
+    full = W.make_inputs(wl)
+    st = W.StreamedInputs(wl, device="cpu")
+    assert st.digest == W.input_digest(full)
+    monkeypatch.setattr(W, "_draw_layer", lambda *a, **k: pytest.fail("layer drawn again"))
+    on = st.to("cpu")
+    for l in range(wl.n_layers):
+        for k in W.LAYER_KEYS:
+            assert torch.equal(on.layers[l][k], full.layers[l][k]), (l, k)
+    assert torch.equal(on.k_cache, full.k_cache) and torch.equal(on.x0, full.x0)
+
+
 def test_every_workload_is_drawn_on_the_cpu_generator():
     assert all(wl.gen_device == "cpu" for wl in W.WORKLOADS.values())
