@@ -404,12 +404,128 @@ __global__ void __launch_bounds__(THREADS, 1)
 // a cluster barrier at the end keeps either CTA from leaving while the other may
 // still touch its shared memory.  A tile's arithmetic is the same fixed-order
 // sum over K as in tc_gemm_kernel.
+// ---------------------------------------------------------------- transposing epilogue
+// One epilogue warp's 32 rows (rows row0 .. row0 + 31, one per lane, as TMEM holds
+// them) x 32 consecutive output columns from col0: the lanes write their rows into
+// a padded 32 x 33 staging block in shared memory, then read it back across rows, so
+// each global load and store covers whole row segments (fp32: 8 lanes x 16 B = one
+// row's 128 bytes, four rows an instruction; bf16: 4 lanes x 16 B, eight rows) instead
+// of 16 bytes of 32 different rows.  Row stride 33 keeps both directions free of bank
+// conflicts.  Rows at or past m_live are neither read nor written.
+constexpr int kStageStride = 33;
+constexpr int kStageFloats = 32 * kStageStride;
+
+template <bool RESID, bool F32>
+__device__ __forceinline__ void flush_chunk(float* stage, const float (&v)[32], int lane, int row0,
+                                            int m_live, int n_out, int col0, void* g_out,
+                                            const float* g_resid) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stage[lane * kStageStride + j] = v[j];
+  __syncwarp();
+  if (F32) {
+    const int c4 = (lane & 7) * 4;
+    float4 r[8];
+    if (RESID) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int row = row0 + 4 * k + (lane >> 3);
+        if (row < m_live)
+          r[k] = *reinterpret_cast<const float4*>(g_resid + (long long)row * n_out + col0 + c4);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int rr = 4 * k + (lane >> 3);
+      const int row = row0 + rr;
+      if (row >= m_live) continue;
+      const float* sv = stage + rr * kStageStride + c4;
+      float4 x = make_float4(sv[0], sv[1], sv[2], sv[3]);
+      if (RESID) {
+        x.x += r[k].x;
+        x.y += r[k].y;
+        x.z += r[k].z;
+        x.w += r[k].w;
+      }
+      *reinterpret_cast<float4*>((float*)g_out + (long long)row * n_out + col0 + c4) = x;
+    }
+  } else {
+    const int c8 = (lane & 3) * 8;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rr = 8 * k + (lane >> 2);
+      const int row = row0 + rr;
+      if (row >= m_live) continue;
+      const float* sv = stage + rr * kStageStride + c8;
+      *reinterpret_cast<uint4*>((__nv_bfloat16*)g_out + (long long)row * n_out + col0 + c8) =
+          make_uint4(pack_bf16(sv[0], sv[1]), pack_bf16(sv[2], sv[3]), pack_bf16(sv[4], sv[5]),
+                     pack_bf16(sv[6], sv[7]));
+    }
+  }
+  __syncwarp();                 // the block is read before the next chunk overwrites it
+}
+
+// The fused epilogue of one epilogue warp's 32 accumulator rows (this lane's TMEM lane
+// holds row row0 + lane, 256 columns from tbase) for output columns tn * 256 (tn * 128
+// for SwiGLU), through flush_chunk.  Same arithmetic as epilogue_row, which the
+// SwiGLU (and row-max) epilogues still use.
+template <int EPI>
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, void* g_out, const float* g_resid,
+                                              const float2* g_rope, int row0, int m_live, int tn,
+                                              uint32_t tbase, float* stage) {
+  const int lane = threadIdx.x & 31;
+  float v[32], u[32];
+  if (EPI == EPI_RESID_F32 || EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
+    const int n0 = tn * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      tmem_ld32(tbase + c * 32, v);
+      tmem_wait_ld();
+      flush_chunk<EPI == EPI_RESID_F32, EPI != EPI_STORE_BF16>(stage, v, lane, row0, m_live,
+                                                               p.N_out, n0 + c * 32, g_out, g_resid);
+    }
+  } else if (EPI == EPI_SWIGLU_BF16 || EPI == EPI_ROWMAX) {
+    // SwiGLU writes half as many bf16 columns as it reads and was measured faster
+    // row by row (the staging costs more than its stores gain)
+    epilogue_row<EPI>(p, g_out, g_resid, g_rope, row0 + lane, row0 + lane < m_live, tn, tbase);
+  } else if (EPI == EPI_ROPE_BF16) {
+    // rotate-half RoPE inside each head of this tile: column j pairs with j + hd/2
+    const int half = p.head_dim / 2;
+    const int tok = (row0 + lane) % p.T;
+    const float4* cs = reinterpret_cast<const float4*>(g_rope + (long long)tok * half);
+    const int n0 = tn * BN;
+#pragma unroll 1
+    for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
+#pragma unroll 1
+      for (int c = 0; c < half; c += 32) {
+        tmem_ld32(tbase + h0 + c, v);
+        tmem_ld32(tbase + h0 + half + c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float4 r = cs[(c + j) >> 1];   // (cos, sin) of columns c + j and c + j + 1
+          const float x1 = v[j], x2 = u[j], y1 = v[j + 1], y2 = u[j + 1];
+          v[j] = x1 * r.x - x2 * r.y;
+          u[j] = x2 * r.x + x1 * r.y;
+          v[j + 1] = y1 * r.z - y2 * r.w;
+          u[j + 1] = y2 * r.z + y1 * r.w;
+        }
+        flush_chunk<false, false>(stage, v, lane, row0, m_live, p.N_out, n0 + h0 + c, g_out,
+                                  nullptr);
+        flush_chunk<false, false>(stage, u, lane, row0, m_live, p.N_out, n0 + h0 + half + c, g_out,
+                                  nullptr);
+      }
+    }
+  }
+}
+
 constexpr int BM2 = 256;
 constexpr int STAGES2 = 6;
 constexpr int A2_BYTES = 128 * BK * 2;       // this CTA's 128 rows of A: 16 KB
 constexpr int B2_BYTES = 128 * BK * 2;       // this CTA's half of the 256 weight rows: 16 KB
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
-constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// the ring, the barriers, then one transposing-epilogue staging block per epilogue warp
+constexpr int STAGE_OFF2 = STAGES2 * STAGE2_BYTES + 256;
+constexpr int SMEM2_BYTES = STAGE_OFF2 + 4 * kStageFloats * 4 + 1024 /*align*/;
 constexpr uint32_t IDESC2 = idesc_bf16_f32(BM2, BN);
 
 struct SharedTail2 {
@@ -550,6 +666,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
     const int q = warp & 3;
+    float* stage = reinterpret_cast<float*>(smem + STAGE_OFF2) + q * kStageFloats;
     int i = 0;
     for (int t = pair; t < n_tiles; t += n_pairs, ++i) {
       const int acc = i & 1;
@@ -561,10 +678,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tile_coords(p, t, tmg, tn);
       const int gi = tile_group(p, tmg, tm);
       const GemmGroupDev& gr = p_in.grp[gi];
-      const int row = tm * BM2 + (int)rank * 128 + q * 32 + lane;
-      const bool live = row < (gi == 0 ? m_live0 : gr.M);
+      const int row0 = tm * BM2 + (int)rank * 128 + q * 32;
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      epilogue_row<EPI>(p, gr.out, gr.resid, gr.rope_cs, row, live, tn, tbase);
+      epilogue_rows<EPI>(p, gr.out, gr.resid, gr.rope_cs, row0, gi == 0 ? m_live0 : gr.M, tn,
+                         tbase, stage);
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
     }
