@@ -56,9 +56,10 @@ def lib():
     return B.load()
 
 
-# The last workload's GPU inputs and the digest of their host draw: the tests of
-# one workload reuse them instead of drawing 16-64 GB again (one workload held at
-# a time; released when the module ends).
+# Each workload's GPU inputs and the digest of their host draw, drawn once for the
+# module: its tests reuse them instead of drawing 16-64 GB again (all three large
+# workloads together hold about 105 GB of the device's 180; released when the
+# module ends).
 _HELD = {}
 
 
@@ -73,8 +74,6 @@ def inputs_and_digest(name):
     """(the workload's seeded inputs on the GPU, SHA-256 of the host draw); the
     KV cache holds the workload's largest context."""
     if name not in _HELD:
-        _HELD.clear()
-        torch.cuda.empty_cache()
         wl = W.WORKLOADS[name]
         assert wl.gen_device == "cpu"
         if name in STREAMED:
