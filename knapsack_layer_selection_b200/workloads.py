@@ -332,6 +332,15 @@ def _hash_update(h, t: torch.Tensor) -> None:
     h.update(t.numpy().tobytes())
 
 
+def window_digest(ww: Sequence[Dict[str, torch.Tensor]]) -> str:
+    """SHA-256 of window_weights' tensors in draw order (per layer Wk then Wv)."""
+    h = hashlib.sha256()
+    for layer in ww:
+        _hash_update(h, layer["wk"])
+        _hash_update(h, layer["wv"])
+    return h.hexdigest()
+
+
 def input_digest(inp: Inputs) -> str:
     """SHA-256 of every input tensor's bytes, in draw order (weights layer by layer,
     then the K cache, the V cache and x0).  Two draws hold the same values iff

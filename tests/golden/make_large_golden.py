@@ -10,6 +10,11 @@ digest of the inputs so that the GPU machine can confirm it drew the same ones.
 
     python tests/golden/make_large_golden.py llama3_8b_8k
     python tests/golden/make_large_golden.py llama3_8b_32k --ctx 4096
+    python tests/golden/make_large_golden.py llama3_8b_8k --kv window
+
+``--kv window`` solves under the window key/value reading (the oracle's R7w: the
+window positions' keys and values recomputed from each candidate's state through
+Wk/Wv, drawn by ``workloads.window_weights``) and records their digest as well.
 
 The 8B shape at 8k context takes about 25 minutes on eight host cores (OpenBLAS
 fp64) and 30 GB of host memory; the Qwen3-32B shape draws its layers one at a
@@ -18,6 +23,7 @@ time (``StreamedInputs``) and needs about 15 GB.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import os
 import sys
 import time
@@ -34,8 +40,9 @@ from oracle import ks_oracle as O  # noqa: E402
 from tests._util import oracle_model, x0_np  # noqa: E402
 
 
-def golden_path(name: str, ctx: int) -> str:
-    return os.path.join(HERE, f"{name}_ctx{ctx}_full.npz")
+def golden_path(name: str, ctx: int, kv: str = "cache") -> str:
+    tag = "" if kv == "cache" else f"_{kv}"
+    return os.path.join(HERE, f"{name}_ctx{ctx}{tag}_full.npz")
 
 
 def pack_sets(sets, n_items: int) -> np.ndarray:
@@ -54,6 +61,8 @@ def main():
     ap.add_argument("--streamed", action="store_true",
                     help="hold one layer of weights at a time (the 64 GB Qwen3-32B shape)")
     ap.add_argument("--ctx", type=int, default=None, help="context to solve at (default: the workload's)")
+    ap.add_argument("--kv", choices=["cache", "window"], default="cache",
+                    help="the attention's key/value reading (R7 or R7w)")
     ap.add_argument("--out", default=None)
     a = ap.parse_args()
 
@@ -68,25 +77,33 @@ def main():
         digest = W.input_digest(inp)
     print(f"{a.workload}: inputs drawn and hashed in {time.time() - t0:.0f} s, sha256 {digest}",
           flush=True)
+    window_sha = ""
+    if a.kv == "window":
+        if isinstance(inp, W.StreamedInputs):
+            raise SystemExit("the window reading is written for the fully drawn workloads only")
+        ww = W.window_weights(base, device="cpu")
+        window_sha = W.window_digest(ww)
+        inp = dataclasses.replace(inp, layers=[{**L, **x} for L, x in zip(inp.layers, ww)])
 
     om = oracle_model(inp)
     x0 = x0_np(inp)
     t = wl.latencies()
     w = O.quantize_weights(t, wl.n_bins)
     t1 = time.time()
-    ref = O.reference_states(om, x0, wl.ctx)
+    ref = O.reference_states(om, x0, wl.ctx, kv=a.kv)
     print(f"reference chain in {time.time() - t1:.0f} s", flush=True)
     t2 = time.time()
-    orc = O.dp_solve(om, x0, wl.ctx, w, t, wl.gamma_max, ref=ref)
+    orc = O.dp_solve(om, x0, wl.ctx, w, t, wl.gamma_max, ref=ref, kv=a.kv)
     secs = time.time() - t2
     print(f"DP over {len(orc.values)} cells x {wl.n_items} items in {secs:.0f} s; best (b={orc.best_b}, "
           f"gamma={orc.best_gamma}, TPT={orc.best_tpt:.6g}), set {orc.sets[orc.best_b]}", flush=True)
 
-    out = a.out or golden_path(a.workload, wl.ctx)
+    out = a.out or golden_path(a.workload, wl.ctx, a.kv)
     np.savez_compressed(
         out,
         workload=np.array(a.workload), ctx=np.int64(wl.ctx), T=np.int64(wl.T),
-        input_sha256=np.array(digest), seed=np.int64(0),
+        input_sha256=np.array(digest), seed=np.int64(0), kv=np.array(a.kv),
+        window_sha256=np.array(window_sha),
         w=np.asarray(w, np.int32), t=np.asarray(t, np.float64),
         bp=orc.dp.bp.astype(np.uint8), cos_s=orc.dp.cos_s, cos_e=orc.dp.cos_e,
         val=orc.dp.val, valid=orc.dp.valid,

@@ -17,6 +17,7 @@ execution equals the dense solve, and Lemma 4.1 is measured at the 8B shape.
 The 32k workload is also re-solved at 4k, 16k and 32k, reporting how many
 Attention and MLP items the chosen sets skip as the context grows.
 """
+import dataclasses
 import os
 from types import SimpleNamespace
 
@@ -39,6 +40,9 @@ GOLDEN = {("llama3_8b_8k", 8192): "llama3_8b_8k_ctx8192_full.npz",
           ("llama3_8b_32k", 16384): "llama3_8b_32k_ctx16384_full.npz",
           ("llama3_8b_32k", 32768): "llama3_8b_32k_ctx32768_full.npz",
           ("qwen3_32b_16k", 16384): "qwen3_32b_16k_ctx16384_full.npz"}
+# under the window key/value reading (R7w: the window's keys and values recomputed
+# from each candidate state through Wk/Wv)
+GOLDEN_WINDOW = {("llama3_8b_8k", 8192): "llama3_8b_8k_ctx8192_window_full.npz"}
 # the Qwen3-32B shape's 64 GB of weights are drawn one layer at a time
 STREAMED = {"qwen3_32b_16k"}
 GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -87,7 +91,7 @@ def gpu_inputs(name):
     return inputs_and_digest(name)[0]
 
 
-def run(name, ctx=None, inp=None, dedup=False):
+def run(name, ctx=None, inp=None, dedup=False, kv="cache"):
     wl = W.WORKLOADS[name]
     if ctx is not None:
         wl = wl.with_ctx(ctx)
@@ -96,7 +100,7 @@ def run(name, ctx=None, inp=None, dedup=False):
                      wl.rms_eps, wl.rope_base, wl.wdtype)
     t = wl.latencies()
     solver = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, t,
-                      B.params(wl.gamma_max, wl.n_bins, dedup=dedup), keep_cos=True)
+                      B.params(wl.gamma_max, wl.n_bins, dedup=dedup), keep_cos=True, kv=kv)
     solver.solve(inp.x0)
     torch.cuda.synchronize()
     solver.check_status()
@@ -172,6 +176,46 @@ def test_full_grid_and_argmax_match_the_oracle(name, ctx):
               f"{wl.n_items} items; oracle best (b={orc.best_b}, gamma={orc.best_gamma}), GPU best "
               f"(b={int(g['best'][0])}, gamma={int(g['best'][1])}); final reference state vs fp64: "
               f"cos {drift:.7f}; {rep}")
+        reports.append(rep)
+        del solver
+        torch.cuda.empty_cache()
+    for rep in reports:
+        rep.assert_ok()
+
+
+WINDOW_GRID = [k for k in GOLDEN_WINDOW
+               if os.path.exists(os.path.join(GOLDEN_DIR, GOLDEN_WINDOW[k]))]
+
+
+@pytest.mark.parametrize("name,ctx", WINDOW_GRID)
+def test_window_reading_full_grid_matches_the_oracle(name, ctx):
+    """The window key/value reading (R7w) at full size: every cell of the full grid
+    and the TPT argmax against the oracle's kv="window" DP on the same inputs and
+    the same Wk/Wv (both digests checked), dense and distinct-state."""
+    path = os.path.join(GOLDEN_DIR, GOLDEN_WINDOW[(name, ctx)])
+    inp, digest = inputs_and_digest(name)
+    wl0 = W.WORKLOADS[name]
+    z, orc = load_golden(path, wl0.n_items)
+    assert digest == str(z["input_sha256"]) and str(z["kv"]) == "window"
+    ww = W.window_weights(wl0, device="cpu")
+    assert W.window_digest(ww) == str(z["window_sha256"]), \
+        "the window weights drawn here differ from the ones the oracle used"
+    winp = dataclasses.replace(inp, layers=[{**L, **{k: v.to("cuda") for k, v in x.items()}}
+                                            for L, x in zip(inp.layers, ww)])
+    reports = []
+    for dedup in (False, True):
+        wl, _, solver = run(name, ctx=ctx, inp=winp, dedup=dedup, kv="window")
+        assert solver.w == [int(x) for x in z["w"]]
+        g = gpu_arrays(solver)
+        check_invariants(wl, solver, g)
+        rep = compare_solve(orc, g, solver.w, 2e-3, wl.n_items, rows_val_gpu=g["rows"],
+                            check_argmax=True)
+        drift = float(O.meancos(g["ref"][-1][None], z["ref_final"])[0])
+        assert drift > 1 - 1e-3, drift
+        print(f"\n{name} @ ctx {ctx}, window reading{' (distinct states)' if dedup else ''}: "
+              f"{solver.C} cells x {wl.n_items} items; oracle best (b={orc.best_b}, "
+              f"gamma={orc.best_gamma}), GPU best (b={int(g['best'][0])}, gamma={int(g['best'][1])}); "
+              f"final reference state vs fp64: cos {drift:.7f}; {rep}")
         reports.append(rep)
         del solver
         torch.cuda.empty_cache()
