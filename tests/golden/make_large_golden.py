@@ -12,7 +12,9 @@ digest of the inputs so that the GPU machine can confirm it drew the same ones.
     python tests/golden/make_large_golden.py llama3_8b_32k --ctx 4096
     python tests/golden/make_large_golden.py llama3_8b_8k --kv window
 
-``--kv window`` solves under the window key/value reading (the oracle's R7w: the
+``--mode exact`` solves the exact-budget table, and ``--prune-tau`` / ``--skip-cap``
+apply the cosine threshold and the skip cap; ``--kv window`` solves under the
+window key/value reading (the oracle's R7w: the
 window positions' keys and values recomputed from each candidate's state through
 Wk/Wv, drawn by ``workloads.window_weights``) and records their digest as well.
 
@@ -40,8 +42,12 @@ from oracle import ks_oracle as O  # noqa: E402
 from tests._util import oracle_model, x0_np  # noqa: E402
 
 
-def golden_path(name: str, ctx: int, kv: str = "cache") -> str:
+def golden_path(name: str, ctx: int, kv: str = "cache", mode: str = "at_most", tau=None,
+                cap=None) -> str:
     tag = "" if kv == "cache" else f"_{kv}"
+    tag += "" if mode == "at_most" else f"_{mode}"
+    tag += "" if tau is None else f"_tau{tau:g}"
+    tag += "" if cap is None else f"_cap{cap}"
     return os.path.join(HERE, f"{name}_ctx{ctx}{tag}_full.npz")
 
 
@@ -63,6 +69,9 @@ def main():
     ap.add_argument("--ctx", type=int, default=None, help="context to solve at (default: the workload's)")
     ap.add_argument("--kv", choices=["cache", "window"], default="cache",
                     help="the attention's key/value reading (R7 or R7w)")
+    ap.add_argument("--mode", choices=["at_most", "exact"], default="at_most")
+    ap.add_argument("--prune-tau", type=float, default=None)
+    ap.add_argument("--skip-cap", type=int, default=None)
     ap.add_argument("--out", default=None)
     a = ap.parse_args()
 
@@ -93,16 +102,19 @@ def main():
     ref = O.reference_states(om, x0, wl.ctx, kv=a.kv)
     print(f"reference chain in {time.time() - t1:.0f} s", flush=True)
     t2 = time.time()
-    orc = O.dp_solve(om, x0, wl.ctx, w, t, wl.gamma_max, ref=ref, kv=a.kv)
+    orc = O.dp_solve(om, x0, wl.ctx, w, t, wl.gamma_max, ref=ref, kv=a.kv, mode=a.mode,
+                     prune_tau=a.prune_tau, skip_cap=a.skip_cap)
     secs = time.time() - t2
     print(f"DP over {len(orc.values)} cells x {wl.n_items} items in {secs:.0f} s; best (b={orc.best_b}, "
           f"gamma={orc.best_gamma}, TPT={orc.best_tpt:.6g}), set {orc.sets[orc.best_b]}", flush=True)
 
-    out = a.out or golden_path(a.workload, wl.ctx, a.kv)
+    out = a.out or golden_path(a.workload, wl.ctx, a.kv, a.mode, a.prune_tau, a.skip_cap)
     np.savez_compressed(
         out,
         workload=np.array(a.workload), ctx=np.int64(wl.ctx), T=np.int64(wl.T),
         input_sha256=np.array(digest), seed=np.int64(0), kv=np.array(a.kv),
+        mode=np.array(a.mode), prune_tau=np.float64(np.nan if a.prune_tau is None else a.prune_tau),
+        skip_cap=np.int64(-1 if a.skip_cap is None else a.skip_cap),
         window_sha256=np.array(window_sha),
         w=np.asarray(w, np.int32), t=np.asarray(t, np.float64),
         bp=orc.dp.bp.astype(np.uint8), cos_s=orc.dp.cos_s, cos_e=orc.dp.cos_e,

@@ -40,9 +40,14 @@ GOLDEN = {("llama3_8b_8k", 8192): "llama3_8b_8k_ctx8192_full.npz",
           ("llama3_8b_32k", 16384): "llama3_8b_32k_ctx16384_full.npz",
           ("llama3_8b_32k", 32768): "llama3_8b_32k_ctx32768_full.npz",
           ("qwen3_32b_16k", 16384): "qwen3_32b_16k_ctx16384_full.npz"}
-# under the window key/value reading (R7w: the window's keys and values recomputed
-# from each candidate state through Wk/Wv)
-GOLDEN_WINDOW = {("llama3_8b_8k", 8192): "llama3_8b_8k_ctx8192_window_full.npz"}
+# the DP's variants on the 8B shape at 8k, each against its own full-grid golden:
+# file -> (key/value reading, budget mode, cosine threshold tau, skip cap); "window" is
+# R7w (the window's keys and values recomputed from each candidate state through Wk/Wv)
+GOLDEN_VARIANTS = {
+    "llama3_8b_8k_ctx8192_window_full.npz": ("window", "at_most", None, None),
+    "llama3_8b_8k_ctx8192_exact_full.npz": ("cache", "exact", None, None),
+    "llama3_8b_8k_ctx8192_tau0.9_cap256_full.npz": ("cache", "at_most", 0.9, 256),
+}
 # the Qwen3-32B shape's 64 GB of weights are drawn one layer at a time
 STREAMED = {"qwen3_32b_16k"}
 GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -91,7 +96,7 @@ def gpu_inputs(name):
     return inputs_and_digest(name)[0]
 
 
-def run(name, ctx=None, inp=None, dedup=False, kv="cache"):
+def run(name, ctx=None, inp=None, dedup=False, kv="cache", mode="at_most", tau=None, cap=None):
     wl = W.WORKLOADS[name]
     if ctx is not None:
         wl = wl.with_ctx(ctx)
@@ -100,7 +105,8 @@ def run(name, ctx=None, inp=None, dedup=False, kv="cache"):
                      wl.rms_eps, wl.rope_base, wl.wdtype)
     t = wl.latencies()
     solver = B.Solver(m, inp.layers, inp.k_cache, inp.v_cache, wl.ctx, wl.T, t,
-                      B.params(wl.gamma_max, wl.n_bins, dedup=dedup), keep_cos=True, kv=kv)
+                      B.params(wl.gamma_max, wl.n_bins, dedup=dedup, budget_mode=mode, prune_tau=tau,
+                               skip_cap=cap), keep_cos=True, kv=kv)
     solver.solve(inp.x0)
     torch.cuda.synchronize()
     solver.check_status()
@@ -183,39 +189,58 @@ def test_full_grid_and_argmax_match_the_oracle(name, ctx):
         rep.assert_ok()
 
 
-WINDOW_GRID = [k for k in GOLDEN_WINDOW
-               if os.path.exists(os.path.join(GOLDEN_DIR, GOLDEN_WINDOW[k]))]
+VARIANT_GRID = [f for f in GOLDEN_VARIANTS if os.path.exists(os.path.join(GOLDEN_DIR, f))]
 
 
-@pytest.mark.parametrize("name,ctx", WINDOW_GRID)
-def test_window_reading_full_grid_matches_the_oracle(name, ctx):
-    """The window key/value reading (R7w) at full size: every cell of the full grid
-    and the TPT argmax against the oracle's kv="window" DP on the same inputs and
-    the same Wk/Wv (both digests checked), dense and distinct-state."""
-    path = os.path.join(GOLDEN_DIR, GOLDEN_WINDOW[(name, ctx)])
+@pytest.mark.parametrize("fname", VARIANT_GRID)
+def test_variant_full_grid_matches_the_oracle(fname):
+    """A variant of the DP at full size (the window key/value reading R7w, the
+    exact-budget table, cosine pruning with the skip cap): every cell of the full grid
+    and the TPT argmax against the oracle's DP of the same variant on the same inputs
+    (digests checked; the window reading's Wk/Wv too), dense and distinct-state.
+    Validity is integer logic and must match wherever no kept value lies within the
+    near-tie distance of tau."""
+    kv, mode, tau, cap = GOLDEN_VARIANTS[fname]
+    name, ctx = "llama3_8b_8k", 8192
     inp, digest = inputs_and_digest(name)
     wl0 = W.WORKLOADS[name]
-    z, orc = load_golden(path, wl0.n_items)
-    assert digest == str(z["input_sha256"]) and str(z["kv"]) == "window"
-    ww = W.window_weights(wl0, device="cpu")
-    assert W.window_digest(ww) == str(z["window_sha256"]), \
-        "the window weights drawn here differ from the ones the oracle used"
-    winp = dataclasses.replace(inp, layers=[{**L, **{k: v.to("cuda") for k, v in x.items()}}
-                                            for L, x in zip(inp.layers, ww)])
+    z, orc = load_golden(os.path.join(GOLDEN_DIR, fname), wl0.n_items)
+    assert digest == str(z["input_sha256"])
+    # (a golden written before the file recorded its budget mode is an at-most one)
+    assert str(z["kv"]) == kv and (str(z["mode"]) if "mode" in z.files else "at_most") == mode
+    if kv == "window":
+        ww = W.window_weights(wl0, device="cpu")
+        assert W.window_digest(ww) == str(z["window_sha256"]), \
+            "the window weights drawn here differ from the ones the oracle used"
+        inp = dataclasses.replace(inp, layers=[{**L, **{k: v.to("cuda") for k, v in x.items()}}
+                                               for L, x in zip(inp.layers, ww)])
     reports = []
     for dedup in (False, True):
-        wl, _, solver = run(name, ctx=ctx, inp=winp, dedup=dedup, kv="window")
+        wl, _, solver = run(name, ctx=ctx, inp=inp, dedup=dedup, kv=kv, mode=mode, tau=tau,
+                            cap=cap)
         assert solver.w == [int(x) for x in z["w"]]
         g = gpu_arrays(solver)
-        check_invariants(wl, solver, g)
+        if mode == "at_most" and tau is None and cap is None:
+            check_invariants(wl, solver, g)
         rep = compare_solve(orc, g, solver.w, 2e-3, wl.n_items, rows_val_gpu=g["rows"],
-                            check_argmax=True)
+                            check_argmax=True, prune_tau=tau)
         drift = float(O.meancos(g["ref"][-1][None], z["ref_final"])[0])
         assert drift > 1 - 1e-3, drift
-        print(f"\n{name} @ ctx {ctx}, window reading{' (distinct states)' if dedup else ''}: "
-              f"{solver.C} cells x {wl.n_items} items; oracle best (b={orc.best_b}, "
-              f"gamma={orc.best_gamma}), GPU best (b={int(g['best'][0])}, gamma={int(g['best'][1])}); "
-              f"final reference state vs fp64: cos {drift:.7f}; {rep}")
+        valid_o = orc.dp.valid[-1]
+        kept = np.where(orc.dp.bp == 1, orc.dp.cos_e, orc.dp.cos_s)
+        near = tau is not None and bool(
+            (np.abs(np.nan_to_num(kept, nan=np.inf) - tau) < 1e-4).any())
+        if not near:
+            assert np.array_equal(np.isfinite(g["values"]), valid_o)
+        if mode == "exact":
+            for b in np.flatnonzero(valid_o):
+                assert g["used_w"][b] == b
+        if cap is not None:
+            assert np.all(np.isnan(g["values"][:max(0, sum(solver.w) - cap)]))
+        print(f"\n{fname}{' (distinct states)' if dedup else ''}: {solver.C} cells x "
+              f"{wl.n_items} items, {int((~valid_o).sum())} final cells invalid; oracle best "
+              f"(b={orc.best_b}, gamma={orc.best_gamma}), GPU best (b={int(g['best'][0])}, "
+              f"gamma={int(g['best'][1])}); final reference state vs fp64: cos {drift:.7f}; {rep}")
         reports.append(rep)
         del solver
         torch.cuda.empty_cache()
